@@ -1,0 +1,168 @@
+"""CPU oracle for two-sided (Kronecker-factored) GPTQ.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  It shares no code with the CUDA library
+(``two_sided_gptq_02_b200``) and never calls it; the product never imports it.
+
+Contents
+  * ``kron_gptq_oracle.c`` (built to ``_build/liboracle.so``): float64 textbook prepare,
+    the naive entry-by-entry two-sided GPTQ (the definition), one-sided GPTQ, RTN and
+    the trace-form proxy loss.
+  * ``literal.py``: the literal (mn) x (mn) vectorized GPTQ on kron(A_d, B_d) for tiny
+    sizes, the LAPACK (numpy) form of prepare, and the certificate checker.
+  * ``parity.py``: comparison of a candidate's codes with the oracle under the
+    boundary rule (a decision taken at a rounding tie is absorbed and counted).
+
+Parity status of each function (what pins it, in tests/test_oracle_pins.py):
+  prepare         pinned: numpy LAPACK Cholesky/inverse, U^T U A_d = I, Kronecker
+                  factor identity, log-determinant identity.
+  quantize_naive  pinned: literal vectorized form (4x4, 6x5, ...), A=B=I and diagonal
+                  factors reduce to RTN, B=I reduces to one-sided GPTQ, A=I reduces to
+                  one-sided GPTQ of W^T, transpose symmetry, leading-block invariance,
+                  loss identity, error bound, certificate.
+  quantize_onesided  pinned: the vectorized form with B=I, RTN when A is diagonal.
+  loss            pinned: closed forms (sum E^2) and numpy einsum of the definition.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kron_gptq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+NOT_FORCED = -(2 ** 31)
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (plain -O2, no fast-math, no FMA contraction)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            lib.ora_prepare.argtypes = [P, I64, ctypes.c_double, P, P]
+            lib.ora_prepare.restype = ctypes.c_int
+            lib.ora_row_scales.argtypes = [P, I64, I64, ctypes.c_int, P]
+            lib.ora_row_scales.restype = None
+            lib.ora_quantize_naive.argtypes = [P, I64, I64, P, P, P, ctypes.c_int, ctypes.c_int, P,
+                                               ctypes.c_double, P, P, P, P, P]
+            lib.ora_quantize_naive.restype = I64
+            lib.ora_quantize_onesided.argtypes = [P, I64, I64, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
+            lib.ora_quantize_onesided.restype = None
+            lib.ora_rtn.argtypes = [P, I64, I64, P, ctypes.c_int, ctypes.c_int, P, P]
+            lib.ora_rtn.restype = None
+            lib.ora_loss.argtypes = [P, P, P, P, I64, I64]
+            lib.ora_loss.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+class OracleNotPD(ValueError):
+    pass
+
+
+def prepare(A, damp: float, *, return_damped: bool = False):
+    """U with U^T U = (A + damp*mean(diag A)*I)^{-1}, upper triangular (float64)."""
+    A = _f64(A)
+    n = A.shape[0]
+    U = np.zeros((n, n), dtype=np.float64)
+    Ad = np.zeros((n, n), dtype=np.float64)
+    rc = _load().ora_prepare(_ptr(A), n, float(damp), _ptr(U), _ptr(Ad))
+    if rc == -1:
+        raise OracleNotPD("factor is not positive definite")
+    if rc != 0:
+        raise MemoryError("oracle prepare: allocation failed")
+    return (U, Ad) if return_damped else U
+
+
+def row_scales(W, qmax: int):
+    W = _f64(W)
+    m, n = W.shape
+    s = np.zeros(m, dtype=np.float64)
+    _load().ora_row_scales(_ptr(W), m, n, int(qmax), _ptr(s))
+    return s
+
+
+def quantize_naive(W, UA, UB, s, qmin: int, qmax: int, *, forced=None, tol: float = 1e-9):
+    """Two-sided GPTQ by definition.  Returns dict(codes, V, E, t, boundary, n_boundary)."""
+    W, UA, UB, s = _f64(W), _f64(UA), _f64(UB), _f64(s)
+    m, n = W.shape
+    assert UA.shape == (n, n) and UB.shape == (m, m) and s.shape == (m,)
+    codes = np.zeros((m, n), dtype=np.int32)
+    V = np.zeros((m, n), dtype=np.float64)
+    E = np.zeros((m, n), dtype=np.float64)
+    t = np.zeros((m, n), dtype=np.float64)
+    bflag = np.zeros((m, n), dtype=np.uint8)
+    f = None
+    if forced is not None:
+        f = np.ascontiguousarray(forced, dtype=np.int32)
+        assert f.shape == (m, n)
+    nb = _load().ora_quantize_naive(_ptr(W), m, n, _ptr(UA), _ptr(UB), _ptr(s), int(qmin), int(qmax),
+                                    _ptr(f), float(tol), _ptr(codes), _ptr(V), _ptr(E), _ptr(t), _ptr(bflag))
+    if nb < 0:
+        raise MemoryError("oracle quantize: allocation failed")
+    return dict(codes=codes, V=V, E=E, t=t, boundary=bflag.astype(bool), n_boundary=int(nb))
+
+
+def quantize_onesided(W, U, S, qmin: int, qmax: int):
+    """Standard GPTQ with per-entry scale S (m x n).  Returns dict(codes, V, E)."""
+    W, U, S = _f64(W), _f64(U), _f64(S)
+    m, n = W.shape
+    codes = np.zeros((m, n), dtype=np.int32)
+    V = np.zeros((m, n), dtype=np.float64)
+    E = np.zeros((m, n), dtype=np.float64)
+    _load().ora_quantize_onesided(_ptr(W), m, n, _ptr(U), _ptr(S), int(qmin), int(qmax),
+                                  _ptr(codes), _ptr(V), _ptr(E))
+    return dict(codes=codes, V=V, E=E)
+
+
+def rtn(W, S, qmin: int, qmax: int):
+    W, S = _f64(W), _f64(S)
+    m, n = W.shape
+    codes = np.zeros((m, n), dtype=np.int32)
+    V = np.zeros((m, n), dtype=np.float64)
+    _load().ora_rtn(_ptr(W), m, n, _ptr(S), int(qmin), int(qmax), _ptr(codes), _ptr(V))
+    return dict(codes=codes, V=V)
+
+
+def loss(W, V, Ad, Bd) -> float:
+    W, V, Ad, Bd = _f64(W), _f64(V), _f64(Ad), _f64(Bd)
+    m, n = W.shape
+    return float(_load().ora_loss(_ptr(W), _ptr(V), _ptr(Ad), _ptr(Bd), m, n))
+
+
+from .literal import (  # noqa: E402,F401
+    certificate,
+    damped,
+    literal_vec,
+    prepare_lapack,
+)
+from .parity import compare_with_oracle  # noqa: E402,F401
