@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Two-sided GPTQ throughput on B200: weights/s and ms per layer, with roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload sq4096] [--dtype f32|f64]
+    python bench.py --impl reference ...      # the CPU oracle on host cores (bounded sample)
+
+One step = one kron_gptq_quantize solve (all sweep + update kernels) of one synthetic layer
+whose inputs (W, U_A, U_B, scales) are already resident in HBM.  Factor preparation is
+untimed, as in the pages' timings of the core solve.  With N GPUs (torchrun, one process per
+GPU) each rank solves its own independently seeded layer: the solve does not shard, so the
+ranks are replicas and `value` is the total weights/s over all ranks (weak scaling).
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "two-sided GPTQ weights/s & ms/layer (4096x4096, 3-bit) + % of roofline"
+TILE = 64
+# B200: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (max SM clock)
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+TF32_OVER_BF16_NOMINAL = 1.1 / 2.25
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="sq4096")
+    ap.add_argument("--dtype", choices=["f32", "f64"], default="f32")
+    ap.add_argument("--damp", type=float, default=0.01)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "MEASURED_PEAKS.json"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="kg_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---------------------------------------------------------------------------------------------- helpers
+def _push_flops(m, n):
+    """FLOPs the trailing-update kernels perform per solve: each (source tile, target tile)
+    pair of the row chain and of the column chain is one 64^3 multiply-add block."""
+    Mt, Nt = math.ceil(m / TILE), math.ceil(n / TILE)
+    pairs = Mt * Nt * (Nt - 1) // 2 + Nt * Mt * (Mt - 1) // 2
+    return 2.0 * TILE ** 3 * pairs
+
+
+def _measure_dgemm_tflops(torch, dev):
+    n = 8192
+    a = torch.randn(n, n, dtype=torch.float64, device=dev)
+    b = torch.randn(n, n, dtype=torch.float64, device=dev)
+    for _ in range(2):
+        a @ b
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        a @ b
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) / 1e3)
+    del a, b
+    return 2.0 * n ** 3 / best / 1e12
+
+
+def _cpu_baseline(spec, W, A, B, damp, budget_s=12.0):
+    """The naive oracle (single thread, plain C) on the leading block of the same layer."""
+    import numpy as np
+
+    import oracle
+    k = 320
+    mb, nb = min(k, spec.m), min(k, spec.n)
+    Wb = W[:mb, :nb].cpu().double().numpy()
+    UA = oracle.prepare(A[:nb, :nb].cpu().double().numpy(), damp)
+    UB = oracle.prepare(B[:mb, :mb].cpu().double().numpy(), damp)
+    s = oracle.row_scales(Wb, spec.qmax)
+    times = []
+    t_start = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oracle.quantize_naive(Wb, UA, UB, s, spec.qmin, spec.qmax)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > budget_s or len(times) >= 8:
+            break
+    t = statistics.median(times)
+    return {"value": mb * nb / t, "unit": "weights/s", "cores": 1, "kind": "oracle",
+            "sample": f"leading {mb}x{nb} block of {spec.name} (its own leading blocks of A, B), naive "
+                      f"O(m^2 n^2) oracle, median of {len(times)} runs of {t:.2f} s; the full "
+                      f"{spec.m}x{spec.n} layer scales by (mn)^2 (extrapolated {t * (spec.m * spec.n / (mb * nb)) ** 2:.3g} s)"}
+
+
+# ---------------------------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import torch  # noqa: F401
+
+    from synth_inputs.layers import layer_inputs, workload
+    spec = workload(args.workload)[0]
+    W, A, B = layer_inputs(spec, device="cpu", leading=320)
+    import oracle
+    oracle.build()
+    for _ in range(args.warmup):
+        _cpu_baseline(spec, W, A, B, args.damp, budget_s=0.0)
+    t0 = time.perf_counter()
+    vals = []
+    for _ in range(args.steps):
+        vals.append(_cpu_baseline(spec, W, A, B, args.damp, budget_s=0.0))
+    el = time.perf_counter() - t0
+    v = statistics.median(x["value"] for x in vals)
+    line = {"metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "m": spec.m, "n": spec.n, "bits": spec.bits,
+                       "sample": vals[0]["sample"]},
+            "cpu_baseline": {"value": v, "unit": "weights/s", "cores": 1, "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import two_sided_gptq_02_b200 as kg
+    from synth_inputs.layers import LayerSpec, layer_inputs, workload
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    base = workload(args.workload)[0]
+    spec = LayerSpec(**{**base.__dict__, "seed": base.seed + 7919 * rank})
+    dt = torch.float32 if args.dtype == "f32" else torch.float64
+    W, A, B = layer_inputs(spec, device=dev)
+    UA, UB, UA32, UB32 = kg.kron_gptq_prepare(A, B, args.damp)
+    if dt == torch.float32:
+        Wd, UAd, UBd = W.float().contiguous(), UA32, UB32
+    else:
+        Wd, UAd, UBd = W, UA, UB
+    sd = kg.kron_gptq_row_scales(Wd, spec.qmax)
+    q = kg.Quantizer(spec.m, spec.n, dt, dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        q.run(Wd, UAd, UBd, sd, spec.qmin, spec.qmax)
+    st = q.status()
+    if st != 0:
+        raise kg.KGError(st, "warm-up solve")
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    kg.kron_gptq_profile_read(reset=True)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+    with ClockSampler(gpu_id) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            q.run(Wd, UAd, UBd, sd, spec.qmin, spec.qmax)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1)
+    counts = kg.kron_gptq_profile_read(reset=True)
+    gpu_launches = sum(v[0] for v in counts.values())
+    st = q.status()
+    if st != 0:
+        raise kg.KGError(st, "timed solve")
+    ms_max = max_over_ranks(ms)
+    clocks = clk.summary()
+    weights = spec.m * spec.n
+    value = world * args.steps * weights / (ms_max / 1e3)
+    ms_per_step = ms_max / args.steps
+
+    # ---- per-kernel durations (separate pass with event timing of every launch)
+    kg.kron_gptq_profile_enable(True)
+    nprof = 3
+    for _ in range(nprof):
+        q.run(Wd, UAd, UBd, sd, spec.qmin, spec.qmax)
+    torch.cuda.synchronize()
+    prof = kg.kron_gptq_profile_read(reset=True)
+    kg.kron_gptq_profile_enable(False)
+
+    peaks, peak_src = _peaks()
+    hbm = float(peaks["hbm_gbs"])
+    fp64_peak = _measure_dgemm_tflops(torch, dev)
+    tf32_peak = float(peaks["bf16_tflops"]) * TF32_OVER_BF16_NOMINAL
+    es = 4 if dt == torch.float32 else 8
+    m, n = spec.m, spec.n
+    graded_flops = 2.0 * m * n * (m + n)
+    bytes_compulsory = es * (2 * m * n + n * n + m * m + m) + m * n
+    if dt == torch.float32:
+        p_tensor, p_name = tf32_peak / 3.0, f"TF32/3 (3xTF32): {peak_src} bf16 burst x 1.1/2.25 / 3"
+    else:
+        p_tensor, p_name = fp64_peak, "FP64: cuBLAS DGEMM 8192^3 measured in this run (burst)"
+    t_roof = max(graded_flops / (p_tensor * 1e12), bytes_compulsory / (hbm * 1e9))
+    solve = {"roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step, "graded_flops": graded_flops,
+             "triangular_flops": graded_flops / 2, "p_tensor_tflops": p_tensor, "p_tensor": p_name,
+             "compulsory_bytes": bytes_compulsory}
+
+    # dominant kernel: the trailing-update (push) kernels
+    pl, pms = prof["push"]
+    ll, lms = prof["leaf"]
+    il, ims = prof["init"]
+    push_flops_per_launch = _push_flops(m, n) / (pl / nprof)
+    push_avg_s = pms / pl / 1e3
+    achieved = push_flops_per_launch / push_avg_s / 1e12
+    if dt == torch.float32:
+        rl = {"bound": "alu", "achieved": achieved, "peak": FP32_SIMT_PEAK_TFLOPS, "unit": "TFLOP/s",
+              "frac": achieved / FP32_SIMT_PEAK_TFLOPS, "traffic": None,
+              "kernel": "k_push_f32", "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}
+    else:
+        rl = {"bound": "tensor", "achieved": achieved, "peak": fp64_peak, "unit": "TFLOP/s",
+              "frac": achieved / fp64_peak, "traffic": None, "kernel": "k_push_f64",
+              "peak_source": "cuBLAS DGEMM measured in this run"}
+    breakdown = {"push_ms_per_solve": pms / nprof, "leaf_ms_per_solve": lms / nprof, "init_ms_per_solve": ims / nprof,
+                 "push_launches_per_solve": pl // nprof, "leaf_launches_per_solve": ll // nprof,
+                 "note": "separate pass with CUDA events around every launch"}
+
+    # ---- end to end: host buffers through the same public call
+    e2e = None
+    if not args.no_e2e:
+        hW = Wd.cpu().pin_memory()
+        hUA, hUB, hs = UAd.cpu().pin_memory(), UBd.cpu().pin_memory(), sd.cpu().pin_memory()
+        dW, dUA, dUB, ds = torch.empty_like(Wd), torch.empty_like(UAd), torch.empty_like(UBd), torch.empty_like(sd)
+        hcodes = torch.empty(m, n, dtype=torch.int8).pin_memory()
+        ke = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            dW.copy_(hW, non_blocking=True)
+            dUA.copy_(hUA, non_blocking=True)
+            dUB.copy_(hUB, non_blocking=True)
+            ds.copy_(hs, non_blocking=True)
+            q.run(dW, dUA, dUB, ds, spec.qmin, spec.qmax)
+            hcodes.copy_(q.codes, non_blocking=True)
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_e2e = max_over_ranks(f0.elapsed_time(f1))
+        e2e = {"value": world * ke * weights / (t_e2e / 1e3), "unit": "weights/s",
+               "h2d_bytes_per_step": int(hW.numel() * es + hUA.numel() * es + hUB.numel() * es + hs.numel() * es),
+               "d2h_bytes_per_step": int(hcodes.numel()), "ms_per_step": t_e2e / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = _cpu_baseline(spec, W, A, B, args.damp)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+                "config": {"workload": f"{args.workload}: {m}x{n} (out x in), {spec.bits}-bit grid "
+                                       f"[{spec.qmin},{spec.qmax}], per-row scale, damp {args.damp}",
+                           "m": m, "n": n, "bits": spec.bits, "solve_dtype": args.dtype,
+                           "parallelism": f"replicas x{world} (independent layers, no collective)",
+                           "l2": "inputs larger than L2 (W, U_A, U_B and a 3-buffer workspace: "
+                                 f"{(bytes_compulsory + 3 * m * n * es) / 1e6:.0f} MB)"},
+                "roofline": rl, "solve_roofline": solve, "kernel_breakdown": breakdown,
+                "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
+                "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
+                          "source": peak_src}}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = _args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

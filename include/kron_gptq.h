@@ -1,0 +1,178 @@
+/*
+ * kron_gptq.h -- C ABI of the two-sided (Kronecker-factored) GPTQ library for NVIDIA B200.
+ *
+ * The library rounds one weight matrix W (m x n; row i = output channel, column j = input
+ * channel) onto a per-row scaled integer grid, minimizing the proxy loss
+ *     D_{A,B} = || B^{1/2} (V - W) A^{1/2} ||_F^2 = vec(V-W)^T (A (x) B) vec(V-W)
+ * with the two-sided GPTQ rounding rule (Babai nearest plane on vec(W) under the Gram matrix
+ * A (x) B).  Sources, by page title and section:
+ *   - "FastKron: Efficient Quantization with Kronecker-Factored Hessians" (later "BaKron"),
+ *     Section 2.1 (notation, quantize instead of round, clipping), Section 2.2 (the
+ *     vectorized algorithm and D_{A,B}), Sections 2.3-2.5 (anti-diagonal parallelism and the
+ *     recursive divide-and-conquer that give O(m+n) steps and O(mn(m+n)) work), Section 2.6
+ *     (inverse and Cholesky as a separate step).
+ *   - "WaterKron and FlipFlop Hessian ...", Section 2 (Notation: Cholesky, RevCholesky,
+ *     damping), Section 2.1 (the scaled integer alphabet).
+ *   - "GPTQ-2D: Cubic-Time Two-Sided Adaptive Rounding" (abstract): the same rounded matrix.
+ *
+ * Conventions for every call:
+ *   - All matrices are dense, row-major, contiguous, in DEVICE memory owned by the caller.
+ *     The library never allocates or frees device memory: each call takes a caller-owned
+ *     workspace of at least the size the matching *_workspace_size() function returns.
+ *   - Calls are asynchronous on the given CUDA stream (passed as void*, a cudaStream_t;
+ *     NULL = the legacy default stream).  Errors the host can see (bad arguments,
+ *     unsupported options, a failed launch) are returned at once and nothing is launched
+ *     after them.  Errors only the device can see (a factor that is not positive definite,
+ *     non-finite input, a device wait that ran out) are written to a status word inside the
+ *     workspace; kron_gptq_sync_status() synchronizes the stream and returns it.
+ *   - Concurrent calls on different streams need distinct workspaces.
+ *   - Status codes: 0 = success, negative = error (see kg_status).
+ */
+#ifndef KRON_GPTQ_H
+#define KRON_GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KG_API __attribute__((visibility("default")))
+#else
+#define KG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kg_status {
+    KG_OK = 0,
+    KG_ERR_ARG = -1,          /* null pointer, negative size, bad grid, misaligned pointer */
+    KG_ERR_UNSUPPORTED = -2,  /* dtype or grid the library does not implement */
+    KG_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
+    KG_ERR_WORKSPACE = -4,    /* workspace smaller than *_workspace_size() */
+    KG_ERR_NOT_PD = -5,       /* (device) a Cholesky pivot was not positive */
+    KG_ERR_NONFINITE = -6,    /* (device) NaN/Inf in W, in the scales or in a factor diagonal */
+    KG_ERR_TIMEOUT = -7       /* (device) a bounded device-side wait ran out */
+} kg_status;
+
+typedef enum kg_dtype {
+    KG_F32 = 1,   /* float32: the solve runs in fp32 with 3xTF32 tensor-core updates */
+    KG_F64 = 2    /* float64: the exact path, fp64 throughout */
+} kg_dtype;
+
+/* Quantization grid: codes are integers in [qmin, qmax] (qmin < 0 < qmax, both within
+ * int8), the value of a code c in row i is row_scale[i] * c.  row_scale is a device array
+ * of m entries with the dtype of the solve ("WaterKron", Section 2.1: V = beta alpha^T (.) Z
+ * with per-row beta and alpha = 1; "FastKron", Section 2.1: integers may be clipped). */
+typedef struct kg_grid {
+    int qmin;
+    int qmax;
+    const void* row_scale;
+} kg_grid;
+
+/* Library version (major*10000 + minor*100 + patch). */
+KG_API int kron_gptq_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+KG_API const char* kron_gptq_status_string(int status);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_prepare -- factors for the solver.
+ *   For each of A (n x n, input side) and B (m x m, output side):
+ *     A_d = A + damp * mean(diag A) * I             (damping, "WaterKron" Sec. 2 Notation)
+ *     U_A = upper-triangular factor with U_A^T U_A = A_d^{-1}
+ *   U_A equals RevCholesky(A_d)^{-T}; its transpose is the lower Cholesky factor of
+ *   A_d^{-1} that the error feedback of "FastKron" Sec. 2.4 uses.  Computed in fp64 by a
+ *   reversed blocked Cholesky of A_d and a blocked triangular inverse.
+ * Arguments:
+ *   A, B      device, symmetric positive (semi)definite, row-major; dtype fac_dtype
+ *             (KG_F32 is promoted to fp64).  The full matrix is read; only its lower
+ *             triangle enters the factorization (symmetry is assumed, not checked).
+ *   n, m      sizes (>= 1).  B may be NULL with m >= 1 to skip the output side.
+ *   damp      relative damping (>= 0); pass 0 if A, B are already damped.
+ *   U_A, U_B  device outputs, fp64, n x n and m x m; the strictly lower triangle is zeroed.
+ *   U_A32, U_B32  optional fp32 copies of the same factors (NULL to skip).
+ *   ws        device workspace of kron_gptq_prepare_workspace_size(max(n, m)) bytes,
+ *             256-byte aligned.
+ * Device errors: KG_ERR_NOT_PD when a pivot of A_d or B_d is not positive (the outputs are
+ *   then unspecified), KG_ERR_NONFINITE for NaN/Inf input.
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_prepare_workspace_size(int64_t k);
+KG_API int kron_gptq_prepare(const void* A, int64_t n, const void* B, int64_t m, int fac_dtype,
+                             double damp, double* U_A, double* U_B, float* U_A32, float* U_B32,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_quantize -- two-sided GPTQ rounding of W ("FastKron" Sec. 2.2-2.5).
+ *   Produces the codes of the naive algorithm: entries visited in any order consistent with
+ *   "top-left first"; for entry (i,j) with current value x:
+ *       c = clamp(rint(x / s_i), qmin, qmax),  Q = s_i c,
+ *       E_ij = (x - Q) / (U_B[i,i] U_A[j,j]),
+ *       W[i',j'] -= U_B[i,i'] E_ij U_A[j,j']   for i' >= i, j' >= j, (i',j') != (i,j).
+ *   Computed as a sweep over anti-diagonals of 64x64 tiles with recursive divide-and-
+ *   conquer batching of the trailing updates over ranges of tile anti-diagonals.
+ *   Rounding is round-half-to-even; in fp64 the codes equal the definition's except at
+ *   entries whose pre-rounding value lies within rounding noise of a half-integer.
+ * Arguments:
+ *   W         device, m x n, dtype (KG_F32 or KG_F64); not modified.
+ *   U_A, U_B  device, n x n and m x m upper-triangular factors (as from prepare), dtype
+ *             matching the solve (the fp32 copies for KG_F32).  Lower triangles are ignored.
+ *   grid      qmin/qmax with -128 <= qmin < 0 < qmax <= 127; row_scale: device, m entries
+ *             of dtype, each finite and > 0 (kron_gptq_row_scales computes max|W_i|/qmax).
+ *   out_codes device, m x n int8.
+ *   out_V     device, m x n, dtype: V = row_scale[i] * code.
+ *   out_E     optional device, m x n, dtype: the scaled errors E (NULL to skip).  They
+ *             satisfy V - W = -U_B^T E U_A and sum(E^2) = D_{A_d,B_d}.
+ *   ws        kron_gptq_quantize_workspace_size(m, n, dtype) bytes, 256-byte aligned.
+ * m == 0 or n == 0 is a no-op returning KG_OK.
+ * Device errors: KG_ERR_NONFINITE (NaN/Inf in W or scales, non-positive scale or factor
+ *   diagonal), KG_ERR_TIMEOUT (a bounded wait in the persistent kernel ran out).
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_quantize_workspace_size(int64_t m, int64_t n, int dtype);
+KG_API int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype,
+                       const void* U_A, const void* U_B, kg_grid grid,
+                       int8_t* out_codes, void* out_V, void* out_E,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_loss -- proxy loss D_{A_d,B_d} = tr((V - W) A_d (V - W)^T B_d)
+ *   = vec(V-W)^T (A_d (x) B_d) vec(V-W)   ("FastKron" Sec. 2.2), accumulated in fp64.
+ *   A_d, B_d are damped exactly as in prepare (same damp).  For the output of quantize it
+ *   equals the sum of E^2 up to rounding.
+ * Arguments: W, V device m x n of dtype; A (n x n), B (m x m) device, dtype fac_dtype;
+ *   out_loss device pointer to one double; ws of kron_gptq_loss_workspace_size(m, n) bytes.
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_loss_workspace_size(int64_t m, int64_t n);
+KG_API int kron_gptq_loss(const void* W, const void* V, int64_t m, int64_t n, int dtype,
+                   const void* A, const void* B, int fac_dtype, double damp,
+                   double* out_loss, void* ws, size_t ws_bytes, void* stream);
+
+/* Per-row scales s_i = max_j |W_ij| / qmax (1 for an all-zero row), chosen from the
+ * original W before any update ("WaterKron" Sec. 2.4: scales are chosen up front).
+ * W device m x n of dtype; out_scale device, m entries of dtype. */
+KG_API int kron_gptq_row_scales(const void* W, int64_t m, int64_t n, int dtype, int qmax,
+                         void* out_scale, void* stream);
+
+/* Synchronize `stream` and return the device status word of the call that used `ws`
+ * (KG_OK or a negative device error), or KG_ERR_CUDA if the synchronization failed. */
+KG_API int kron_gptq_sync_status(const void* ws, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Diagnostics (tracing).  The library counts every kernel launch by kind:
+ *   0 init/validation, 1 in-tile sweep (leaf), 2 trailing band update (push),
+ *   3 factor preparation, 4 loss and scales, 5 persistent whole-solve kernel.
+ * kron_gptq_profile_enable(1) additionally brackets each launch with a pair of CUDA events
+ * recorded on the launch's own stream (the events are host-side resources; no device
+ * memory is allocated).  kron_gptq_profile_read() waits for the recorded events, adds
+ * their elapsed times per kind, and copies the counters (launches[k], ms[k] for
+ * k < nkinds; either pointer may be NULL); reset != 0 clears them afterwards.
+ * Not meant for production timing loops: the events add host work per launch.
+ * --------------------------------------------------------------------------------------- */
+KG_API void kron_gptq_profile_enable(int enable);
+KG_API int kron_gptq_profile_read(int64_t* launches, double* ms, int nkinds, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRON_GPTQ_H */

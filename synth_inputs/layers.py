@@ -78,12 +78,14 @@ def workload(name: str) -> list[LayerSpec]:
     return WORKLOADS[name]
 
 
-def _gram(gen: torch.Generator, k: int, N: int, sigma: float, device) -> torch.Tensor:
+def _gram(gen: torch.Generator, k: int, N: int, sigma: float, device, lead: int | None = None) -> torch.Tensor:
     Z = torch.randn(N, k, generator=gen, dtype=torch.float64)
     Mn = torch.randn(k, k, generator=gen, dtype=torch.float64)
     s = torch.exp(sigma * torch.randn(k, generator=gen, dtype=torch.float64))
     Mm = Mn.mul_(0.1 / math.sqrt(k))
     Mm.diagonal().add_(s)
+    if lead is not None:
+        Mm = Mm[:, :lead]          # the leading block of X^T X needs only these columns of X
     X = Z.to(device) @ Mm.to(device)
     del Z, Mm
     G = X.T @ X
@@ -91,21 +93,29 @@ def _gram(gen: torch.Generator, k: int, N: int, sigma: float, device) -> torch.T
     return 0.5 * (G + G.T)   # exact symmetry
 
 
-def layer_inputs(spec: LayerSpec, device="cpu", *, with_factors: bool = True):
-    """Return (W, A, B) as float64 tensors on ``device`` (A: n x n, B: m x m)."""
+def layer_inputs(spec: LayerSpec, device="cpu", *, with_factors: bool = True, leading: int | None = None):
+    """Return (W, A, B) as float64 tensors on ``device`` (A: n x n, B: m x m).
+
+    ``leading=k`` returns only W[:k,:k], A[:k,:k], B[:k,:k] -- the same values as the full
+    layer's leading blocks (same draws), without forming the full Gram products.
+    """
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(spec.seed))
     W = torch.randn(spec.m, spec.n, generator=gen, dtype=torch.float64) / math.sqrt(spec.n)
     mask = torch.rand(spec.m, spec.n, generator=gen, dtype=torch.float64) < spec.outlier_frac
     W = torch.where(mask, W * 10.0, W)
+    if leading is not None:
+        W = W[:leading, :leading].contiguous()
     W = W.to(device)
     if not with_factors:
         return W, None, None
-    A = _gram(gen, spec.n, spec.n_samples, spec.sigma_in, device)
+    la = None if leading is None else min(leading, spec.n)
+    lb = None if leading is None else min(leading, spec.m)
+    A = _gram(gen, spec.n, spec.n_samples, spec.sigma_in, device, la)
     if spec.identity_B:
-        B = torch.eye(spec.m, dtype=torch.float64, device=device)
+        B = torch.eye(spec.m if lb is None else lb, dtype=torch.float64, device=device)
     else:
-        B = _gram(gen, spec.m, spec.n_samples, spec.sigma_out, device)
+        B = _gram(gen, spec.m, spec.n_samples, spec.sigma_out, device, lb)
     return W, A, B
 
 

@@ -296,3 +296,13 @@ def test_planted_mistakes_fail_a_pin(mutation):
     cert = oracle.certificate(*args[:3], f["s"], f["qmin"], f["qmax"], c, V, E)
     caught = (not np.array_equal(c, lit["codes"])) or cert["resid_rel"] > 1e-9 or cert["code_mismatch"] > 0
     assert caught, mutation
+
+
+def test_generator_leading_block_is_consistent():
+    from synth_inputs.layers import LayerSpec, layer_inputs
+    spec = LayerSpec(name="t", m=48, n=40, seed=5, n_samples=64, outlier_frac=0.05)
+    W, A, B = layer_inputs(spec)
+    Wl, Al, Bl = layer_inputs(spec, leading=16)
+    assert np.array_equal(W[:16, :16].numpy(), Wl.numpy())
+    np.testing.assert_allclose(A[:16, :16].numpy(), Al.numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(B[:16, :16].numpy(), Bl.numpy(), rtol=1e-12, atol=1e-14)

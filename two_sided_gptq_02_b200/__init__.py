@@ -1,0 +1,36 @@
+"""Two-sided (Kronecker-factored) GPTQ on NVIDIA B200 -- Python binding.
+
+Thin ctypes binding of the C ABI in ``include/kron_gptq.h`` (library ``libkrongptq.so``,
+built in-tree by ``python -m two_sided_gptq_02_b200.build``).  Every step of the solve runs
+in the library's CUDA kernels; this module only marshals arguments.  PyTorch provides
+device memory and streams.  There is no CPU fallback: if the library is missing the import
+of the binding fails with an error that says how to build it.
+
+Public functions mirror the C names:
+    kron_gptq_prepare(A, B, damp)          -> U_A, U_B (fp64) and fp32 copies
+    kron_gptq_quantize(W, U_A, U_B, ...)   -> codes (int8), V, E
+    kron_gptq_loss(W, V, A, B, damp)       -> float
+    kron_gptq_row_scales(W, qmax)          -> per-row scales
+    kron_gptq_sync_status(ws, stream)      -> device status word
+"""
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    KG_F32,
+    KG_F64,
+    KGError,
+    Quantizer,
+    PROFILE_KINDS,
+    kron_gptq_loss,
+    kron_gptq_profile_enable,
+    kron_gptq_profile_read,
+    kron_gptq_prepare,
+    kron_gptq_quantize,
+    kron_gptq_row_scales,
+    kron_gptq_status_string,
+    kron_gptq_sync_status,
+    kron_gptq_version,
+    lib_path,
+    load_library,
+    quantize_workspace_bytes,
+)

@@ -1,0 +1,237 @@
+"""ctypes binding of libkrongptq.so (see include/kron_gptq.h for the contract)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+KG_F32 = 1
+KG_F64 = 2
+_ERRORS = {
+    -1: "KG_ERR_ARG", -2: "KG_ERR_UNSUPPORTED", -3: "KG_ERR_CUDA", -4: "KG_ERR_WORKSPACE",
+    -5: "KG_ERR_NOT_PD", -6: "KG_ERR_NONFINITE", -7: "KG_ERR_TIMEOUT",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lock = threading.Lock()
+_lib = None
+
+
+class KGError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        self.name = _ERRORS.get(self.code, "KG_ERR_UNKNOWN")
+        super().__init__(f"{where}: {self.name} ({self.code})")
+
+
+class _Grid(ctypes.Structure):
+    _fields_ = [("qmin", ctypes.c_int), ("qmax", ctypes.c_int), ("row_scale", ctypes.c_void_p)]
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libkrongptq.so")
+
+
+def load_library():
+    """Load the CUDA library; raise ImportError (no fallback) if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = lib_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m two_sided_gptq_02_b200.build` "
+                              "(there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        L.kron_gptq_version.restype = I
+        L.kron_gptq_status_string.argtypes = [I]
+        L.kron_gptq_status_string.restype = ctypes.c_char_p
+        L.kron_gptq_prepare_workspace_size.argtypes = [I64]
+        L.kron_gptq_prepare_workspace_size.restype = SZ
+        L.kron_gptq_prepare.argtypes = [P, I64, P, I64, I, ctypes.c_double, P, P, P, P, P, SZ, P]
+        L.kron_gptq_prepare.restype = I
+        L.kron_gptq_quantize_workspace_size.argtypes = [I64, I64, I]
+        L.kron_gptq_quantize_workspace_size.restype = SZ
+        L.kron_gptq_quantize.argtypes = [P, I64, I64, I, P, P, _Grid, P, P, P, P, SZ, P]
+        L.kron_gptq_quantize.restype = I
+        L.kron_gptq_loss_workspace_size.argtypes = [I64, I64]
+        L.kron_gptq_loss_workspace_size.restype = SZ
+        L.kron_gptq_loss.argtypes = [P, P, I64, I64, I, P, P, I, ctypes.c_double, P, P, SZ, P]
+        L.kron_gptq_loss.restype = I
+        L.kron_gptq_row_scales.argtypes = [P, I64, I64, I, I, P, P]
+        L.kron_gptq_row_scales.restype = I
+        L.kron_gptq_sync_status.argtypes = [P, P]
+        L.kron_gptq_sync_status.restype = I
+        L.kron_gptq_profile_enable.argtypes = [I]
+        L.kron_gptq_profile_enable.restype = None
+        L.kron_gptq_profile_read.argtypes = [P, P, I, I]
+        L.kron_gptq_profile_read.restype = I
+        _lib = L
+        return L
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KG_F32
+    if t.dtype == torch.float64:
+        return KG_F64
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or float64)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major)")
+
+
+def _raise(rc: int, where: str):
+    if rc != 0:
+        raise KGError(rc, where)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # the caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+PROFILE_KINDS = ("init", "leaf", "push", "prepare", "loss", "solve")
+
+
+def kron_gptq_profile_enable(enable: bool) -> None:
+    load_library().kron_gptq_profile_enable(1 if enable else 0)
+
+
+def kron_gptq_profile_read(reset: bool = False) -> dict:
+    """{kind: (launches, milliseconds)}; waits for the recorded events."""
+    n = len(PROFILE_KINDS)
+    launches = (ctypes.c_int64 * n)()
+    ms = (ctypes.c_double * n)()
+    _raise(load_library().kron_gptq_profile_read(ctypes.cast(launches, ctypes.c_void_p),
+                                                 ctypes.cast(ms, ctypes.c_void_p), n, 1 if reset else 0),
+           "kron_gptq_profile_read")
+    return {k: (int(launches[i]), float(ms[i])) for i, k in enumerate(PROFILE_KINDS)}
+
+
+def kron_gptq_version() -> int:
+    return load_library().kron_gptq_version()
+
+
+def kron_gptq_status_string(code: int) -> str:
+    return load_library().kron_gptq_status_string(int(code)).decode()
+
+
+def kron_gptq_sync_status(ws: torch.Tensor, stream=None) -> int:
+    return load_library().kron_gptq_sync_status(_ptr(ws), _stream(stream))
+
+
+def kron_gptq_prepare(A: torch.Tensor, B: torch.Tensor | None, damp: float, *, fp32_copies: bool = True,
+                      stream=None, check: bool = True):
+    """U_A (n x n) and U_B (m x m), upper triangular, U^T U = (X + damp*mean(diag X)*I)^{-1}.
+
+    Returns (U_A, U_B, U_A32, U_B32); U_B* are None when B is None.
+    """
+    L = load_library()
+    _check_dev(A, B)
+    n = A.shape[0]
+    m = B.shape[0] if B is not None else 0
+    if B is not None and B.dtype != A.dtype:
+        raise TypeError("A and B must share a dtype")
+    dev = A.device
+    UA = torch.empty(n, n, dtype=torch.float64, device=dev)
+    UB = torch.empty(m, m, dtype=torch.float64, device=dev) if B is not None else None
+    UA32 = torch.empty(n, n, dtype=torch.float32, device=dev) if fp32_copies else None
+    UB32 = torch.empty(m, m, dtype=torch.float32, device=dev) if (fp32_copies and B is not None) else None
+    ws = _workspace(L.kron_gptq_prepare_workspace_size(max(n, m)), dev)
+    rc = L.kron_gptq_prepare(_ptr(A), n, _ptr(B), m, _dtype_code(A), float(damp), _ptr(UA), _ptr(UB),
+                             _ptr(UA32), _ptr(UB32), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "kron_gptq_prepare")
+    if check:
+        _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_prepare (device)")
+    return UA, UB, UA32, UB32
+
+
+def quantize_workspace_bytes(m: int, n: int, dtype: torch.dtype) -> int:
+    code = KG_F64 if dtype == torch.float64 else KG_F32
+    return int(load_library().kron_gptq_quantize_workspace_size(int(m), int(n), code))
+
+
+class Quantizer:
+    """Reusable workspace and outputs for repeated solves of one shape (no allocation per call)."""
+
+    def __init__(self, m: int, n: int, dtype: torch.dtype, device, *, want_E: bool = False):
+        self.m, self.n, self.dtype = int(m), int(n), dtype
+        self.code = KG_F64 if dtype == torch.float64 else KG_F32
+        L = load_library()
+        self.ws = _workspace(L.kron_gptq_quantize_workspace_size(self.m, self.n, self.code), device)
+        self.codes = torch.empty(self.m, self.n, dtype=torch.int8, device=device)
+        self.V = torch.empty(self.m, self.n, dtype=dtype, device=device)
+        self.E = torch.empty(self.m, self.n, dtype=dtype, device=device) if want_E else None
+
+    def run(self, W, U_A, U_B, row_scale, qmin: int, qmax: int, stream=None) -> None:
+        """Enqueue one solve on `stream`; does not synchronize."""
+        L = load_library()
+        for t in (W, U_A, U_B, row_scale):
+            if t.dtype != self.dtype:
+                raise TypeError("W, U_A, U_B and row_scale must all have the solve dtype")
+        _check_dev(W, U_A, U_B, row_scale)
+        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or U_B.shape != (self.m, self.m) \
+                or row_scale.shape != (self.m,):
+            raise ValueError("shape mismatch")
+        grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
+        rc = L.kron_gptq_quantize(_ptr(W), self.m, self.n, self.code, _ptr(U_A), _ptr(U_B), grid,
+                                  _ptr(self.codes), _ptr(self.V), _ptr(self.E), _ptr(self.ws), self.ws.numel(),
+                                  _stream(stream))
+        _raise(rc, "kron_gptq_quantize")
+
+    def status(self, stream=None) -> int:
+        return kron_gptq_sync_status(self.ws, stream)
+
+
+def kron_gptq_quantize(W, U_A, U_B, qmin: int, qmax: int, row_scale, *, want_E: bool = False, stream=None,
+                       check: bool = True):
+    """Two-sided GPTQ of W.  Returns (codes int8, V, E or None)."""
+    q = Quantizer(W.shape[0], W.shape[1], W.dtype, W.device, want_E=want_E)
+    q.run(W, U_A, U_B, row_scale, qmin, qmax, stream=stream)
+    if check:
+        _raise(q.status(stream), "kron_gptq_quantize (device)")
+    return q.codes, q.V, q.E
+
+
+def kron_gptq_loss(W, V, A, B, damp: float, *, stream=None) -> float:
+    """tr((V-W) A_d (V-W)^T B_d) with A_d, B_d damped as in prepare (fp64 accumulation)."""
+    L = load_library()
+    _check_dev(W, V, A, B)
+    m, n = W.shape
+    out = torch.zeros(1, dtype=torch.float64, device=W.device)
+    ws = _workspace(L.kron_gptq_loss_workspace_size(m, n), W.device)
+    rc = L.kron_gptq_loss(_ptr(W), _ptr(V), m, n, _dtype_code(W), _ptr(A), _ptr(B), _dtype_code(A), float(damp),
+                          _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "kron_gptq_loss")
+    _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_loss (device)")
+    return float(out.item())
+
+
+def kron_gptq_row_scales(W, qmax: int, *, stream=None):
+    L = load_library()
+    _check_dev(W)
+    m, n = W.shape
+    s = torch.empty(m, dtype=W.dtype, device=W.device)
+    _raise(L.kron_gptq_row_scales(_ptr(W), m, n, _dtype_code(W), int(qmax), _ptr(s), _stream(stream)),
+           "kron_gptq_row_scales")
+    return s

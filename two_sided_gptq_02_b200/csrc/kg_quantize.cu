@@ -1,0 +1,496 @@
+// kg_quantize.cu -- two-sided GPTQ rounding (FastKron / BaKron) on 64x64 tiles.
+//
+// Algorithm ("FastKron: Efficient Quantization with Kronecker-Factored Hessians",
+// Sections 2.2-2.5).  Entry (i,j) is rounded once every entry to its top-left has pushed
+// its error; the error E_ij = (x - Q)/(U_B[i,i] U_A[j,j]) reaches entry (i',j') as
+// U_B[i,i'] E_ij U_A[j,j'] (i' >= i, j' >= j).  The update factors through two chains,
+// which is the associativity of the batched update W -= U_B^T E U_A (Section 2.4):
+//     row chain     R[i,j] = sum_{j'<j} E[i,j'] U_A[j',j]          (along a row)
+//                   X[i,j] = R[i,j] + E[i,j] U_A[j,j]              (complete once (i,j) is done)
+//     column chain  C[i,j] = sum_{i'<i} U_B[i',i] X[i',j]          (down a column)
+//     x_ij = W_ij - C_ij - U_B[i,i] R_ij .
+// Only complete values are pushed (E along rows, X down columns), so every source/target
+// pair costs one multiply-add and the total work is mn(m+n)/2 multiply-adds whatever the
+// batching.
+//
+// Tiles.  W is cut into 64x64 tiles; tile (I,J) lies on tile anti-diagonal D = I + J.
+// Tiles of one tile anti-diagonal are independent (Section 2.3).  The schedule is the
+// recursion of Section 2.5 applied to ranges of tile anti-diagonals:
+//     solve(D0, D1): if one diagonal: leaf(D0)
+//                    else solve(D0, mid); push(D0 | mid | D1); solve(mid, D1)
+// leaf(D)  -- every tile on D runs the in-tile anti-diagonal sweep (one CTA per tile);
+// push     -- the band of tiles [D0, mid) sends its errors to the band [mid, D1): for each
+//             target tile (I,J) in [mid, D1)
+//               R[I,J]  += sum_{J': I+J' in [D0,mid)} E[I,J'] U_A[J',J]       (row chain)
+//               W~[I,J] -= sum_{I': I'+J in [D0,mid)} U_B[I',I]^T X[I',J]     (column chain)
+//             Both are dense GEMMs over contiguous K ranges.
+#include <algorithm>
+
+#include "kg_common.cuh"
+#include "kg_gemm.cuh"
+#include "kg_profile.cuh"
+
+namespace kg {
+
+constexpr int T = KG_T;
+
+// ---------------------------------------------------------------------------------------
+// Workspace layout (all offsets 256-byte aligned):
+//   [status 256B][Wt Mp*Np][R Mp*Np][E Mp*Np][scale Mp][UApad Np*Np][UBpad Mp*Mp]
+// Wt holds W minus the column chain, R holds the row chain and, once a tile is solved, its
+// complete X.  The padded factors exist only when m or n is not a multiple of 64; the pad
+// is the identity, so padded entries have zero error and never touch real ones.
+// ---------------------------------------------------------------------------------------
+struct QLayout {
+    int64_t m, n, Mt, Nt, Mp, Np;
+    bool padded;
+    size_t es;
+    size_t off_wt, off_r, off_e, off_s, off_ua, off_ub, total;
+};
+
+static QLayout q_layout(int64_t m, int64_t n, size_t es) {
+    QLayout L{};
+    L.m = m; L.n = n; L.es = es;
+    L.Mt = ceil_div(m, T); L.Nt = ceil_div(n, T);
+    L.Mp = L.Mt * T; L.Np = L.Nt * T;
+    L.padded = (L.Mp != m) || (L.Np != n);
+    size_t off = kStatusBytes;
+    L.off_wt = off; off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
+    L.off_r = off;  off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
+    L.off_e = off;  off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
+    L.off_s = off;  off = align_up(off + (size_t)L.Mp * es, 256);
+    L.off_ua = off;
+    if (L.padded) {
+        off = align_up(off + (size_t)(L.Np * L.Np) * es, 256);
+        L.off_ub = off;
+        off = align_up(off + (size_t)(L.Mp * L.Mp) * es, 256);
+    } else {
+        L.off_ub = off;
+    }
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------------------------ init
+template <typename Real>
+__global__ void k_init_w(const Real* __restrict__ W, int64_t m, int64_t n, int64_t Np, int64_t Mp,
+                         Real* __restrict__ Wt, Real* __restrict__ R, DevStatus* st) {
+    const int64_t total = Mp * Np;
+    for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < total; p += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = p / Np, j = p % Np;
+        Real v = Real(0);
+        if (i < m && j < n) {
+            v = W[i * n + j];
+            if (!isfinite(v)) set_status(st, KG_ERR_NONFINITE, (int)(i * n + j));
+        }
+        Wt[p] = v;
+        R[p] = Real(0);
+    }
+}
+
+template <typename Real>
+__global__ void k_init_scale(const Real* __restrict__ s, int64_t m, int64_t Mp, Real* __restrict__ sp,
+                             DevStatus* st) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < Mp; i += (int64_t)gridDim.x * blockDim.x) {
+        Real v = Real(1);
+        if (i < m) {
+            v = s[i];
+            if (!isfinite(v) || !(v > Real(0))) { set_status(st, KG_ERR_NONFINITE, (int)i); v = Real(1); }
+        }
+        sp[i] = v;
+    }
+}
+
+// Copy an upper-triangular factor into a padded buffer with identity padding, zeroing the
+// strictly lower triangle; also validates the diagonal.
+template <typename Real>
+__global__ void k_pad_factor(const Real* __restrict__ U, int64_t k, int64_t kp, Real* __restrict__ Up,
+                             DevStatus* st) {
+    const int64_t total = kp * kp;
+    for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < total; p += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = p / kp, c = p % kp;
+        Real v = Real(0);
+        if (r < k && c < k) {
+            if (c >= r) v = U[r * k + c];
+        } else if (r == c) {
+            v = Real(1);
+        }
+        Up[p] = v;
+    }
+}
+
+template <typename Real>
+__global__ void k_check_diag2(const Real* __restrict__ UA, int64_t n, const Real* __restrict__ UB, int64_t m,
+                              DevStatus* st) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n || i < m; i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < n) {
+            const Real d = UA[i * n + i];
+            if (!isfinite(d) || !(d > Real(0))) set_status(st, KG_ERR_NONFINITE, (int)i);
+        }
+        if (i < m) {
+            const Real d = UB[i * m + i];
+            if (!isfinite(d) || !(d > Real(0))) set_status(st, KG_ERR_NONFINITE, (int)i);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------ leaf
+// One CTA per tile (I, D-I) of tile anti-diagonal D.  256 threads: four per tile row.
+//
+// In-tile problem: w' = W~[I,J] - U_B[I,I]^T R[I,J] (the external row chain enters through
+// the diagonal block of U_B), then two-sided GPTQ on the 64x64 tile with factors
+// a = U_A[J,J], b = U_B[I,I], swept anti-diagonal by anti-diagonal:
+//     r_ij = sum_{j'<j} E_ij' a[j',j],   c_ij = sum_{i'<i} b[i',i] X_i'j,
+//     x = w'_ij - c_ij - b_ii r_ij,  c = clamp(rint(x/s_i)),  Q = s_i c,
+//     E_ij = (x - Q)/(b_ii a_jj),   X_ij = r_ij + E_ij a_jj.
+// The complete X of the tile is R[I,J] + X (stored back into R for the column chain).
+template <typename Real>
+struct LeafSmem {
+    static constexpr int S = T + 4;   // row stride: quad-strided reads are bank-conflict free
+    Real aT[T][S];    // aT[j][j'] = a[j'][j]
+    Real bT[T][S];    // bT[i][i'] = b[i'][i]
+    Real Es[T][S];    // errors, row-major
+    Real XT[T][S];    // local X, transposed: XT[j][i]
+    Real Ws[T][S];    // w', then Q
+    Real Rs[T][S];    // external row chain R[I,J]
+    Real s[T], invs[T], inva[T], invb[T];
+    int8_t Cs[T][T];
+};
+
+template <typename Real>
+__global__ void __launch_bounds__(256)
+k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
+       Real* __restrict__ Wt, Real* __restrict__ R, Real* __restrict__ Ebuf,
+       const Real* __restrict__ UA, int64_t ldA, const Real* __restrict__ UB, int64_t ldB,
+       const Real* __restrict__ sp, int qmin, int qmax,
+       int8_t* __restrict__ codes, Real* __restrict__ V, Real* __restrict__ outE) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    LeafSmem<Real>& sm = *reinterpret_cast<LeafSmem<Real>*>(smem_raw);
+    const int Imin = max(0, D - Nt + 1);
+    const int I = Imin + blockIdx.x;
+    const int J = D - I;
+    const int tid = threadIdx.x;
+    const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
+
+    // ---- load tiles
+    for (int idx = tid; idx < T * T; idx += 256) {
+        const int r = idx / T, c = idx % T;
+        const Real av = UA[(c0 + r) * ldA + c0 + c];     // a[r][c]
+        const Real bv = UB[(r0 + r) * ldB + r0 + c];     // b[r][c]
+        sm.aT[c][r] = (c >= r) ? av : Real(0);
+        sm.bT[c][r] = (c >= r) ? bv : Real(0);
+        sm.Ws[r][c] = Wt[(r0 + r) * Np + c0 + c];
+        sm.Rs[r][c] = R[(r0 + r) * Np + c0 + c];
+        sm.Es[r][c] = Real(0);
+        sm.XT[r][c] = Real(0);
+    }
+    if (tid < T) {
+        const Real s = sp[r0 + tid];
+        sm.s[tid] = s;
+        sm.invs[tid] = Real(1) / s;
+    }
+    __syncthreads();
+    if (tid < T) {
+        sm.inva[tid] = Real(1) / sm.aT[tid][tid];
+        sm.invb[tid] = Real(1) / sm.bT[tid][tid];
+    }
+
+    // ---- w' = W~ - b^T R   (triangular: b^T[i][k] = 0 for k > i)
+    {
+        const int ty = tid >> 4, tx = tid & 15;
+        Real acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = Real(0);
+        const int kmax = ty * 4 + 3;
+        for (int k = 0; k <= kmax; ++k) {
+            Real bv[4], rv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) bv[a] = sm.bT[ty * 4 + a][k];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) rv[b] = sm.Rs[k][tx * 4 + b];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] += bv[a] * rv[b];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) sm.Ws[ty * 4 + a][tx * 4 + b] -= acc[a][b];
+    }
+    __syncthreads();
+
+    // ---- anti-diagonal sweep
+    const int i = tid >> 2, q = tid & 3;
+    const Real bii = sm.bT[i][i];
+    const Real fqmin = Real(qmin), fqmax = Real(qmax);
+    for (int d = 0; d < 2 * T - 1; ++d) {
+        const int j = d - i;
+        const bool active = (j >= 0) && (j < T);
+        Real c = Real(0), r = Real(0);
+        if (active) {
+            for (int k = q; k < i; k += 4) c += sm.bT[i][k] * sm.XT[j][k];
+            for (int k = q; k < j; k += 4) r += sm.Es[i][k] * sm.aT[j][k];
+        }
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        c += __shfl_xor_sync(0xffffffffu, c, 2);
+        r += __shfl_xor_sync(0xffffffffu, r, 1);
+        r += __shfl_xor_sync(0xffffffffu, r, 2);
+        if (active && q == 0) {
+            const Real x = sm.Ws[i][j] - c - bii * r;
+            Real code = rint(x * sm.invs[i]);
+            code = code < fqmin ? fqmin : (code > fqmax ? fqmax : code);
+            const Real Qv = code * sm.s[i];
+            const Real e = (x - Qv) * sm.invb[i] * sm.inva[j];
+            sm.Es[i][j] = e;
+            sm.XT[j][i] = r + e * sm.aT[j][j];
+            sm.Ws[i][j] = Qv;
+            sm.Cs[i][j] = (int8_t)code;
+        }
+        __syncthreads();
+    }
+
+    // ---- write back
+    for (int idx = tid; idx < T * T; idx += 256) {
+        const int r = idx / T, c = idx % T;
+        const int64_t gi = r0 + r, gj = c0 + c;
+        R[gi * Np + gj] = sm.Rs[r][c] + sm.XT[c][r];
+        Ebuf[gi * Np + gj] = sm.Es[r][c];
+        if (gi < m && gj < n) {
+            codes[gi * n + gj] = sm.Cs[r][c];
+            V[gi * n + gj] = sm.Ws[r][c];
+            if (outE) outE[gi * n + gj] = sm.Es[r][c];
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------ push
+// Grid: x = position along a target diagonal, y = target diagonal offset from mid,
+// z = chain (0: row chain into R, 1: column chain into W~).
+__global__ void __launch_bounds__(Dmma64::kThreads)
+k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
+           double* __restrict__ Wt, double* __restrict__ R, const double* __restrict__ E,
+           const double* __restrict__ UA, int64_t ldA, const double* __restrict__ UB, int64_t ldB) {
+    __shared__ Dmma64::Smem sm;
+    const int D = mid + blockIdx.y;
+    const int I = max(0, D - Nt + 1) + blockIdx.x;
+    if (I > min(D, Mt - 1)) return;
+    const int J = D - I;
+    Dmma64::Acc acc;
+    Dmma64::zero(acc);
+    if (blockIdx.z == 0) {
+        const int k0 = max(0, D0 - I), k1 = min(Nt, mid - I);
+        if (k0 >= k1) return;
+        LdA_RowMajor64 la{E + (int64_t)I * T * Np + (int64_t)k0 * T, Np};
+        LdB_RowMajor64 lb{UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA};
+        Dmma64::run(acc, sm, (k1 - k0) * T, la, lb);
+        double* out = R + (int64_t)I * T * Np + (int64_t)J * T;
+        Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] += v; });
+    } else {
+        const int k0 = max(0, D0 - J), k1 = min(Mt, mid - J);
+        if (k0 >= k1) return;
+        LdA_Trans64 la{UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB};
+        LdB_RowMajor64 lb{R + (int64_t)k0 * T * Np + (int64_t)J * T, Np};
+        Dmma64::run(acc, sm, (k1 - k0) * T, la, lb);
+        double* out = Wt + (int64_t)I * T * Np + (int64_t)J * T;
+        Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] -= v; });
+    }
+}
+
+__global__ void __launch_bounds__(Simt64f::kThreads)
+k_push_f32(int D0, int mid, int Mt, int Nt, int64_t Np,
+           float* __restrict__ Wt, float* __restrict__ R, const float* __restrict__ E,
+           const float* __restrict__ UA, int64_t ldA, const float* __restrict__ UB, int64_t ldB) {
+    __shared__ __align__(16) Simt64f::Smem sm;
+    const int D = mid + blockIdx.y;
+    const int I = max(0, D - Nt + 1) + blockIdx.x;
+    if (I > min(D, Mt - 1)) return;
+    const int J = D - I;
+    Simt64f::Acc acc;
+    Simt64f::zero(acc);
+    if (blockIdx.z == 0) {
+        const int k0 = max(0, D0 - I), k1 = min(Nt, mid - I);
+        if (k0 >= k1) return;
+        LdAf_RowMajor la{E + (int64_t)I * T * Np + (int64_t)k0 * T, Np};
+        LdBf_RowMajor lb{UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA};
+        Simt64f::run(acc, sm, (k1 - k0) * T, la, lb);
+        float* out = R + (int64_t)I * T * Np + (int64_t)J * T;
+        Simt64f::for_each(acc, [&](int r, int c, float v) { out[(int64_t)r * Np + c] += v; });
+    } else {
+        const int k0 = max(0, D0 - J), k1 = min(Mt, mid - J);
+        if (k0 >= k1) return;
+        LdAf_Trans la{UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB};
+        LdBf_RowMajor lb{R + (int64_t)k0 * T * Np + (int64_t)J * T, Np};
+        Simt64f::run(acc, sm, (k1 - k0) * T, la, lb);
+        float* out = Wt + (int64_t)I * T * Np + (int64_t)J * T;
+        Simt64f::for_each(acc, [&](int r, int c, float v) { out[(int64_t)r * Np + c] -= v; });
+    }
+}
+
+// ------------------------------------------------------------------------------ driver
+template <typename Real>
+struct QArgs {
+    QLayout L;
+    Real *Wt, *R, *E, *sp;
+    const Real *UA, *UB;
+    int64_t ldA, ldB;
+    int qmin, qmax;
+    int8_t* codes;
+    Real* V;
+    Real* outE;
+    cudaStream_t st;
+};
+
+template <typename Real>
+static int launch_leaf(const QArgs<Real>& a, int D) {
+    const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
+    const int Imin = std::max(0, D - Nt + 1), Imax = std::min(D, Mt - 1);
+    const int ntiles = Imax - Imin + 1;
+    const size_t smem = sizeof(LeafSmem<Real>);
+    ProfScope ps(PK_LEAF, a.st);
+    k_leaf<Real><<<ntiles, 256, smem, a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA,
+                                              a.UB, a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
+    KG_LAUNCH_CHECK();
+    return KG_OK;
+}
+
+static int launch_push(const QArgs<double>& a, int D0, int mid, int D1) {
+    const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
+    dim3 grid(std::min(Mt, Nt), D1 - mid, 2);
+    ProfScope ps(PK_PUSH, a.st);
+    k_push_f64<<<grid, Dmma64::kThreads, 0, a.st>>>(D0, mid, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB, a.ldB);
+    KG_LAUNCH_CHECK();
+    return KG_OK;
+}
+static int launch_push(const QArgs<float>& a, int D0, int mid, int D1) {
+    const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
+    dim3 grid(std::min(Mt, Nt), D1 - mid, 2);
+    ProfScope ps(PK_PUSH, a.st);
+    k_push_f32<<<grid, Simt64f::kThreads, 0, a.st>>>(D0, mid, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB, a.ldB);
+    KG_LAUNCH_CHECK();
+    return KG_OK;
+}
+
+template <typename Real>
+static int solve_range(const QArgs<Real>& a, int D0, int D1) {
+    if (D1 - D0 == 1) return launch_leaf(a, D0);
+    const int mid = (D0 + D1) / 2;
+    int rc = solve_range(a, D0, mid);
+    if (rc) return rc;
+    rc = launch_push(a, D0, mid, D1);
+    if (rc) return rc;
+    return solve_range(a, mid, D1);
+}
+
+template <typename Real>
+static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, const void* UB_, kg_grid grid,
+                         int8_t* codes, void* V, void* outE, void* ws, size_t ws_bytes, cudaStream_t st) {
+    const QLayout L = q_layout(m, n, sizeof(Real));
+    if (ws_bytes < L.total) return KG_ERR_WORKSPACE;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    DevStatus* status = reinterpret_cast<DevStatus*>(base);
+    QArgs<Real> a;
+    a.L = L;
+    a.Wt = reinterpret_cast<Real*>(base + L.off_wt);
+    a.R = reinterpret_cast<Real*>(base + L.off_r);
+    a.E = reinterpret_cast<Real*>(base + L.off_e);
+    a.sp = reinterpret_cast<Real*>(base + L.off_s);
+    a.qmin = grid.qmin; a.qmax = grid.qmax;
+    a.codes = codes;
+    a.V = static_cast<Real*>(V);
+    a.outE = static_cast<Real*>(outE);
+    a.st = st;
+
+    KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
+    const int nb = 148 * 4;
+    {
+        ProfScope ps(PK_INIT, st);
+        k_init_w<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(W), m, n, L.Np, L.Mp, a.Wt, a.R, status);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_init_scale<Real><<<std::max<int64_t>(1, std::min<int64_t>(nb, ceil_div(L.Mp, 256))), 256, 0, st>>>(
+            static_cast<const Real*>(grid.row_scale), m, L.Mp, a.sp, status);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_check_diag2<Real><<<std::max<int64_t>(1, ceil_div(std::max(m, n), 256)), 256, 0, st>>>(
+            static_cast<const Real*>(UA_), n, static_cast<const Real*>(UB_), m, status);
+    }
+    KG_LAUNCH_CHECK();
+    if (L.padded) {
+        Real* UAp = reinterpret_cast<Real*>(base + L.off_ua);
+        Real* UBp = reinterpret_cast<Real*>(base + L.off_ub);
+        {
+            ProfScope ps(PK_INIT, st);
+            k_pad_factor<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(UA_), n, L.Np, UAp, status);
+        }
+        KG_LAUNCH_CHECK();
+        {
+            ProfScope ps(PK_INIT, st);
+            k_pad_factor<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(UB_), m, L.Mp, UBp, status);
+        }
+        KG_LAUNCH_CHECK();
+        a.UA = UAp; a.ldA = L.Np;
+        a.UB = UBp; a.ldB = L.Mp;
+    } else {
+        a.UA = static_cast<const Real*>(UA_); a.ldA = n;
+        a.UB = static_cast<const Real*>(UB_); a.ldB = m;
+    }
+    return solve_range(a, 0, (int)(L.Mt + L.Nt - 1));
+}
+
+static bool leaf_smem_configured[2] = {false, false};
+
+template <typename Real>
+static int configure_leaf() {
+    const int idx = sizeof(Real) == 8 ? 1 : 0;
+    if (!leaf_smem_configured[idx]) {
+        KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(LeafSmem<Real>)));
+        leaf_smem_configured[idx] = true;
+    }
+    return KG_OK;
+}
+
+}  // namespace kg
+
+using namespace kg;
+
+extern "C" size_t kron_gptq_quantize_workspace_size(int64_t m, int64_t n, int dtype) {
+    if (m < 0 || n < 0) return 0;
+    if (dtype != KG_F32 && dtype != KG_F64) return 0;
+    if (m == 0 || n == 0) return kStatusBytes;
+    return q_layout(m, n, dtype == KG_F64 ? 8 : 4).total;
+}
+
+extern "C" int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype, const void* U_A,
+                                  const void* U_B, kg_grid grid, int8_t* out_codes, void* out_V, void* out_E,
+                                  void* ws, size_t ws_bytes, void* stream) {
+    if (dtype != KG_F32 && dtype != KG_F64) return KG_ERR_UNSUPPORTED;
+    if (m < 0 || n < 0) return KG_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return KG_ERR_ARG;
+    if (grid.qmin >= 0 || grid.qmax <= 0 || grid.qmin < -128 || grid.qmax > 127) return KG_ERR_UNSUPPORTED;
+    if (m > (int64_t)1 << 20 || n > (int64_t)1 << 20) return KG_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m == 0 || n == 0) {
+        if (ws_bytes < kStatusBytes) return KG_ERR_WORKSPACE;
+        KG_CUDA_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+        return KG_OK;
+    }
+    if (!W || !U_A || !U_B || !grid.row_scale || !out_codes || !out_V) return KG_ERR_ARG;
+    if (ws_bytes < q_layout(m, n, dtype == KG_F64 ? 8 : 4).total) return KG_ERR_WORKSPACE;
+    if (dtype == KG_F64) {
+        int rc = configure_leaf<double>();
+        if (rc) return rc;
+        return quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
+    }
+    int rc = configure_leaf<float>();
+    if (rc) return rc;
+    return quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
+}
