@@ -146,7 +146,8 @@ def test_ragged_fp64_full_oracle(kg, m, n, bits, seed):
     codes, V, E = _run(kg, c, spec.qmin, spec.qmax)
     res = _assert_fp64_parity(codes, c["W"], c["UA"], c["UB"], c["s"], spec.qmin, spec.qmax)
     lo = np.sum(res["oracle"]["E"] ** 2)
-    assert abs(np.sum(E ** 2) - lo) <= 1e-9 * max(lo, 1e-300)
+    # when every code reproduces W exactly (e.g. one column) E is pure rounding noise
+    assert abs(np.sum(E ** 2) - lo) <= 1e-9 * lo + 1e-20
 
 
 @pytest.mark.parametrize("m,n", [(127, 129), (200, 70)])
@@ -192,7 +193,8 @@ def test_sq1024_identity_B_equals_onesided(kg, dtype):
     spec = workload("sq1024_onesided")[0]
     W, A, B = _inputs(spec)
     c = _case(W, A, B, spec.qmax, dtype)
-    assert np.array_equal(c["UB"], np.eye(spec.m))
+    # B = I is damped to (1 + damp) I: U_B is diagonal, so there is no coupling across rows
+    assert np.array_equal(c["UB"], np.diag(np.diag(c["UB"])))
     codes, V, E = _run(kg, c, spec.qmin, spec.qmax)
     one = oracle.quantize_onesided(c["W"], c["UA"], np.repeat(c["s"][:, None], spec.n, 1), spec.qmin, spec.qmax)
     agree = np.mean(codes == one["codes"])
