@@ -158,6 +158,34 @@ KG_API int kron_gptq_row_scales(const void* W, int64_t m, int64_t n, int dtype, 
 KG_API int kron_gptq_sync_status(const void* ws, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * kron_gptq_quantize_noalloc -- kron_gptq_quantize without a caller workspace.
+ *   The paper has no counterpart: this is a deployment variant for callers that cannot
+ *   allocate device memory -- code running inside a host framework whose allocator owns all
+ *   device memory and forbids direct cudaMalloc, or a service path that must not allocate
+ *   after start-up (cudaMalloc may synchronize the device).  It runs exactly the same kernels
+ *   as kron_gptq_quantize, with the scratch in a fixed device array of
+ *   KG_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the library holds
+ *   until the process exits.  It allocates nothing: no cudaMalloc, no cudaFree.
+ * Arguments: as kron_gptq_quantize, without ws/ws_bytes, plus
+ *   dev_status  optional device pointer to one int that receives the device status word of
+ *               this call (KG_OK or a negative device error) in stream order; NULL to skip.
+ * Limits and behaviour:
+ *   - Problems whose scratch (kron_gptq_quantize_workspace_size(m, n, dtype)) exceeds
+ *     KG_NOALLOC_SCRATCH_BYTES are rejected with KG_ERR_WORKSPACE before anything is launched
+ *     (about 12 bytes per weight in fp32 and 24 in fp64: fp32 fits e.g. 1536 x 1536, fp64
+ *     e.g. 1024 x 1024).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the one array and each call re-initialises what it reads; calls whose
+ *     executions overlap on the same GPU (different streams, threads) race on it.
+ * --------------------------------------------------------------------------------------- */
+#define KG_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+KG_API int kron_gptq_quantize_noalloc(const void* W, int64_t m, int64_t n, int dtype,
+                                      const void* U_A, const void* U_B, kg_grid grid,
+                                      int8_t* out_codes, void* out_V, void* out_E,
+                                      int* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Diagnostics (tracing).  The library counts every kernel launch by kind:
  *   0 init/validation, 1 in-tile sweep (leaf), 2 trailing band update (push),
  *   3 factor preparation, 4 loss and scales, 5 persistent whole-solve kernel.

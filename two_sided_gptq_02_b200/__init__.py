@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     kron_gptq_profile_read,
     kron_gptq_prepare,
     kron_gptq_quantize,
+    kron_gptq_quantize_noalloc,
     kron_gptq_row_scales,
     kron_gptq_status_string,
     kron_gptq_sync_status,

@@ -65,6 +65,8 @@ def load_library():
         L.kron_gptq_row_scales.restype = I
         L.kron_gptq_sync_status.argtypes = [P, P]
         L.kron_gptq_sync_status.restype = I
+        L.kron_gptq_quantize_noalloc.argtypes = [P, I64, I64, I, P, P, _Grid, P, P, P, P, P]
+        L.kron_gptq_quantize_noalloc.restype = I
         L.kron_gptq_profile_enable.argtypes = [I]
         L.kron_gptq_profile_enable.restype = None
         L.kron_gptq_profile_read.argtypes = [P, P, I, I]
@@ -211,6 +213,20 @@ def kron_gptq_quantize(W, U_A, U_B, qmin: int, qmax: int, row_scale, *, want_E: 
     if check:
         _raise(q.status(stream), "kron_gptq_quantize (device)")
     return q.codes, q.V, q.E
+
+
+def kron_gptq_quantize_noalloc(W, U_A, U_B, qmin: int, qmax: int, row_scale, codes, V, E=None, dev_status=None,
+                               *, stream=None) -> None:
+    """Allocation-free solve into caller-provided outputs (codes int8, V, optional E, optional
+    one-int device status).  The library uses its fixed internal scratch array instead of a
+    workspace; see include/kron_gptq.h for the size limit and the sharing rules."""
+    L = load_library()
+    _check_dev(W, U_A, U_B, row_scale, codes, V, E, dev_status)
+    m, n = W.shape
+    grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
+    rc = L.kron_gptq_quantize_noalloc(_ptr(W), m, n, _dtype_code(W), _ptr(U_A), _ptr(U_B), grid, _ptr(codes),
+                                      _ptr(V), _ptr(E), _ptr(dev_status), _stream(stream))
+    _raise(rc, "kron_gptq_quantize_noalloc")
 
 
 def kron_gptq_loss(W, V, A, B, damp: float, *, stream=None) -> float:

@@ -494,3 +494,76 @@ extern "C" int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype
     if (rc) return rc;
     return quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
 }
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of kron_gptq_quantize.
+//
+// Some callers cannot hand the library a workspace: code that runs inside a host framework
+// whose allocator owns all device memory and forbids direct cudaMalloc, or a service path that
+// must not allocate after start-up (cudaMalloc may synchronize the whole device).  For them the
+// scratch lives in a fixed file-scope device array, KG_NOALLOC_SCRATCH_BYTES large, which every
+// GPU that loads the library keeps until the process exits.  In host code the array's name is
+// only a host-side stand-in, so its device address is fetched with cudaGetSymbolAddress, once
+// per device, with that device current, on the first call made on that device.  All calls share
+// the array: each call re-initialises everything it reads (status word, W~, R, scales), and calls
+// whose executions overlap on a GPU race on it.
+// ---------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace kg {
+
+static_assert(KG_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte alignment");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KG_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+// Device address of the scratch array on the current device (looked up once per device).
+static int noalloc_scratch(void** out) {
+    int dev = -1;
+    KG_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return KG_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KG_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return KG_OK;
+}
+
+}  // namespace kg
+
+extern "C" int kron_gptq_quantize_noalloc(const void* W, int64_t m, int64_t n, int dtype, const void* U_A,
+                                          const void* U_B, kg_grid grid, int8_t* out_codes, void* out_V,
+                                          void* out_E, int* dev_status, void* stream) {
+    if (dtype != KG_F32 && dtype != KG_F64) return KG_ERR_UNSUPPORTED;
+    if (m < 0 || n < 0) return KG_ERR_ARG;
+    if (grid.qmin >= 0 || grid.qmax <= 0 || grid.qmin < -128 || grid.qmax > 127) return KG_ERR_UNSUPPORTED;
+    if (m > (int64_t)1 << 20 || n > (int64_t)1 << 20) return KG_ERR_UNSUPPORTED;
+    const size_t need = (m == 0 || n == 0) ? kStatusBytes : q_layout(m, n, dtype == KG_F64 ? 8 : 4).total;
+    if (need > (size_t)KG_NOALLOC_SCRATCH_BYTES) return KG_ERR_WORKSPACE;
+    if (m != 0 && n != 0 && (!W || !U_A || !U_B || !grid.row_scale || !out_codes || !out_V)) return KG_ERR_ARG;
+    void* scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m == 0 || n == 0) {
+        KG_CUDA_TRY(cudaMemsetAsync(scratch, 0, kStatusBytes, st));
+    } else if (dtype == KG_F64) {
+        rc = configure_leaf<double>();
+        if (!rc) rc = quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, scratch,
+                                            (size_t)KG_NOALLOC_SCRATCH_BYTES, st);
+    } else {
+        rc = configure_leaf<float>();
+        if (!rc) rc = quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, scratch,
+                                           (size_t)KG_NOALLOC_SCRATCH_BYTES, st);
+    }
+    if (rc) return rc;
+    if (dev_status) KG_CUDA_TRY(cudaMemcpyAsync(dev_status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, st));
+    return KG_OK;
+}
