@@ -28,6 +28,7 @@
 
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
+#include "kg_leaf.cuh"
 #include "kg_profile.cuh"
 
 namespace kg {
@@ -130,139 +131,6 @@ __global__ void k_check_diag2(const Real* __restrict__ UA, int64_t n, const Real
         if (i < m) {
             const Real d = UB[i * m + i];
             if (!isfinite(d) || !(d > Real(0))) set_status(st, KG_ERR_NONFINITE, (int)i);
-        }
-    }
-}
-
-// ------------------------------------------------------------------------------ leaf
-// One CTA per tile (I, D-I) of tile anti-diagonal D.  256 threads: four per tile row.
-//
-// In-tile problem: w' = W~[I,J] - U_B[I,I]^T R[I,J] (the external row chain enters through
-// the diagonal block of U_B), then two-sided GPTQ on the 64x64 tile with factors
-// a = U_A[J,J], b = U_B[I,I], swept anti-diagonal by anti-diagonal:
-//     r_ij = sum_{j'<j} E_ij' a[j',j],   c_ij = sum_{i'<i} b[i',i] X_i'j,
-//     x = w'_ij - c_ij - b_ii r_ij,  c = clamp(rint(x/s_i)),  Q = s_i c,
-//     E_ij = (x - Q)/(b_ii a_jj),   X_ij = r_ij + E_ij a_jj.
-// The complete X of the tile is R[I,J] + X (stored back into R for the column chain).
-template <typename Real>
-struct LeafSmem {
-    static constexpr int S = T + 4;   // row stride: quad-strided reads are bank-conflict free
-    Real aT[T][S];    // aT[j][j'] = a[j'][j]
-    Real bT[T][S];    // bT[i][i'] = b[i'][i]
-    Real Es[T][S];    // errors, row-major
-    Real XT[T][S];    // local X, transposed: XT[j][i]
-    Real Ws[T][S];    // w', then Q
-    Real Rs[T][S];    // external row chain R[I,J]
-    Real s[T], invs[T], inva[T], invb[T];
-    int8_t Cs[T][T];
-};
-
-template <typename Real>
-__global__ void __launch_bounds__(256)
-k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
-       Real* __restrict__ Wt, Real* __restrict__ R, Real* __restrict__ Ebuf,
-       const Real* __restrict__ UA, int64_t ldA, const Real* __restrict__ UB, int64_t ldB,
-       const Real* __restrict__ sp, int qmin, int qmax,
-       int8_t* __restrict__ codes, Real* __restrict__ V, Real* __restrict__ outE) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    LeafSmem<Real>& sm = *reinterpret_cast<LeafSmem<Real>*>(smem_raw);
-    const int Imin = max(0, D - Nt + 1);
-    const int I = Imin + blockIdx.x;
-    const int J = D - I;
-    const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
-
-    // ---- load tiles
-    for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
-        const Real av = UA[(c0 + r) * ldA + c0 + c];     // a[r][c]
-        const Real bv = UB[(r0 + r) * ldB + r0 + c];     // b[r][c]
-        sm.aT[c][r] = (c >= r) ? av : Real(0);
-        sm.bT[c][r] = (c >= r) ? bv : Real(0);
-        sm.Ws[r][c] = Wt[(r0 + r) * Np + c0 + c];
-        sm.Rs[r][c] = R[(r0 + r) * Np + c0 + c];
-        sm.Es[r][c] = Real(0);
-        sm.XT[r][c] = Real(0);
-    }
-    if (tid < T) {
-        const Real s = sp[r0 + tid];
-        sm.s[tid] = s;
-        sm.invs[tid] = Real(1) / s;
-    }
-    __syncthreads();
-    if (tid < T) {
-        sm.inva[tid] = Real(1) / sm.aT[tid][tid];
-        sm.invb[tid] = Real(1) / sm.bT[tid][tid];
-    }
-
-    // ---- w' = W~ - b^T R   (triangular: b^T[i][k] = 0 for k > i)
-    {
-        const int ty = tid >> 4, tx = tid & 15;
-        Real acc[4][4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = Real(0);
-        const int kmax = ty * 4 + 3;
-        for (int k = 0; k <= kmax; ++k) {
-            Real bv[4], rv[4];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) bv[a] = sm.bT[ty * 4 + a][k];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) rv[b] = sm.Rs[k][tx * 4 + b];
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] += bv[a] * rv[b];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) sm.Ws[ty * 4 + a][tx * 4 + b] -= acc[a][b];
-    }
-    __syncthreads();
-
-    // ---- anti-diagonal sweep
-    const int i = tid >> 2, q = tid & 3;
-    const Real bii = sm.bT[i][i];
-    const Real fqmin = Real(qmin), fqmax = Real(qmax);
-    for (int d = 0; d < 2 * T - 1; ++d) {
-        const int j = d - i;
-        const bool active = (j >= 0) && (j < T);
-        Real c = Real(0), r = Real(0);
-        if (active) {
-            for (int k = q; k < i; k += 4) c += sm.bT[i][k] * sm.XT[j][k];
-            for (int k = q; k < j; k += 4) r += sm.Es[i][k] * sm.aT[j][k];
-        }
-        c += __shfl_xor_sync(0xffffffffu, c, 1);
-        c += __shfl_xor_sync(0xffffffffu, c, 2);
-        r += __shfl_xor_sync(0xffffffffu, r, 1);
-        r += __shfl_xor_sync(0xffffffffu, r, 2);
-        if (active && q == 0) {
-            const Real x = sm.Ws[i][j] - c - bii * r;
-            Real code = rint(x * sm.invs[i]);
-            code = code < fqmin ? fqmin : (code > fqmax ? fqmax : code);
-            const Real Qv = code * sm.s[i];
-            const Real e = (x - Qv) * sm.invb[i] * sm.inva[j];
-            sm.Es[i][j] = e;
-            sm.XT[j][i] = r + e * sm.aT[j][j];
-            sm.Ws[i][j] = Qv;
-            sm.Cs[i][j] = (int8_t)code;
-        }
-        __syncthreads();
-    }
-
-    // ---- write back
-    for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
-        const int64_t gi = r0 + r, gj = c0 + c;
-        R[gi * Np + gj] = sm.Rs[r][c] + sm.XT[c][r];
-        Ebuf[gi * Np + gj] = sm.Es[r][c];
-        if (gi < m && gj < n) {
-            codes[gi * n + gj] = sm.Cs[r][c];
-            V[gi * n + gj] = sm.Ws[r][c];
-            if (outE) outE[gi * n + gj] = sm.Es[r][c];
         }
     }
 }
