@@ -172,8 +172,9 @@ KG_API int kron_gptq_sync_status(const void* ws, void* stream);
  * Limits and behaviour:
  *   - Problems whose scratch (kron_gptq_quantize_workspace_size(m, n, dtype)) exceeds
  *     KG_NOALLOC_SCRATCH_BYTES are rejected with KG_ERR_WORKSPACE before anything is launched
- *     (about 12 bytes per weight in fp32 and 24 in fp64: fp32 fits e.g. 1536 x 1536, fp64
- *     e.g. 1024 x 1024).
+ *     (for a square layer about 40 bytes per weight in fp32, which keeps split copies of the
+ *     operands for the tensor cores, and 24 in fp64: fp32 fits e.g. 896 x 896, fp64 e.g.
+ *     1024 x 1024).
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream capture.
  *   - All calls share the one array and each call re-initialises what it reads; calls whose

@@ -32,7 +32,7 @@ def kg():
 
 
 @pytest.mark.parametrize("dtype,m,n", [(torch.float64, 300, 200), (torch.float32, 320, 256),
-                                       (torch.float32, 1024, 1024)])
+                                       (torch.float32, 768, 768), (torch.float64, 1024, 1024)])
 def test_noalloc_matches_workspace_entry_point(kg, dtype, m, n):
     spec, (W, A, B) = small_layer(m, n, 17, bits=3)
     W, A, B = W.numpy(), A.numpy(), B.numpy()

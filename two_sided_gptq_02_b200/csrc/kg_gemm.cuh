@@ -142,6 +142,98 @@ struct LdB_Trans64 {
     }
 };
 
+// ------------------------------------------------------------------------------ fp64, pipelined
+// Same warp tiling and mma.sync m8n8k4 f64 as Dmma64, but the operands are plain copies of
+// global memory staged with cp.async (16-byte granules) into two shared-memory stages, so the
+// copy of chunk k+1 overlaps the MMAs of chunk k.
+//   A_KM: A is stored K x 64 (A(r,k) = A[k*lda + r]) instead of 64 x K (A[r*lda + k]).
+//   B_T : B is stored 64 x K (B(k,c) = B[c*ldb + k]) instead of K x 64 (B[k*ldb + c]).
+// All source rows must start on 16-byte boundaries (ld and offsets even).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <bool A_KM, bool B_T>
+struct DmmaPipe {
+    static constexpr int BK = 16, STAGES = 2, kThreads = 128;
+    static constexpr int SR = BK + 4;      // stride of a 64 x BK stage (row per output row/column)
+    static constexpr int SK = 64 + 4;      // stride of a BK x 64 stage (row per k)
+    static constexpr int A_ELEMS = A_KM ? BK * SK : 64 * SR;
+    static constexpr int B_ELEMS = B_T ? 64 * SR : BK * SK;
+    struct Smem {
+        __align__(16) double a[STAGES][A_ELEMS];
+        __align__(16) double b[STAGES][B_ELEMS];
+    };
+
+    __device__ static __forceinline__ void load(Smem& sm, int s, const double* A, int64_t lda, const double* B,
+                                                int64_t ldb, int k0) {
+        const int tid = threadIdx.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {   // 64 x 16 doubles = 512 granules of 16 bytes
+            const int f = e * kThreads + tid;
+            if (!A_KM) {
+                const int r = f >> 3, c = (f & 7) * 2;
+                cp_async16(&sm.a[s][r * SR + c], A + (int64_t)r * lda + k0 + c);
+            } else {
+                const int k = f >> 5, r = (f & 31) * 2;
+                cp_async16(&sm.a[s][k * SK + r], A + (int64_t)(k0 + k) * lda + r);
+            }
+            if (!B_T) {
+                const int k = f >> 5, c = (f & 31) * 2;
+                cp_async16(&sm.b[s][k * SK + c], B + (int64_t)(k0 + k) * ldb + c);
+            } else {
+                const int c = f >> 3, k = (f & 7) * 2;
+                cp_async16(&sm.b[s][c * SR + k], B + (int64_t)c * ldb + k0 + k);
+            }
+        }
+    }
+
+    __device__ static __forceinline__ void run(Dmma64::Acc& acc, Smem& sm, int K, const double* A, int64_t lda,
+                                               const double* B, int64_t ldb) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+        const int nk = K / BK;
+        load(sm, 0, A, lda, B, ldb, 0);
+        cp_async_commit();
+        for (int c = 0; c < nk; ++c) {
+            if (c + 1 < nk) {
+                load(sm, (c + 1) & 1, A, lda, B, ldb, (c + 1) * BK);
+                cp_async_commit();
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();
+            const double* as = sm.a[c & 1];
+            const double* bs = sm.b[c & 1];
+#pragma unroll
+            for (int kk = 0; kk < BK; kk += 4) {
+                double a[4], b[4];
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    const int r = wm + mi * 8 + (lane >> 2), k = kk + (lane & 3);
+                    a[mi] = A_KM ? as[k * SK + r] : as[r * SR + k];
+                }
+#pragma unroll
+                for (int ni = 0; ni < 4; ++ni) {
+                    const int cc = wn + ni * 8 + (lane >> 2), k = kk + (lane & 3);
+                    b[ni] = B_T ? bs[cc * SR + k] : bs[k * SK + cc];
+                }
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni) Dmma64::mma(acc.c[mi][ni][0], acc.c[mi][ni][1], a[mi], b[ni]);
+            }
+            __syncthreads();
+        }
+    }
+};
+
 // ------------------------------------------------------------------------------ fp32
 struct Simt64f {
     static constexpr int BM = 64, BN = 64, BK = 32;

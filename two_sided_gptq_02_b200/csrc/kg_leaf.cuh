@@ -15,12 +15,13 @@
 // step d-1) was computed during step d-1 as pre_x; so the dependent chain of a step is one
 // shared-memory load, two FMAs and the rounding.  The dot products for column j+1 run in the
 // shadow of that chain: lanes read 16-byte chunks interleaved across the quad (k = VW*q +
-// 4*VW*t + u), which with a row stride of 16 (mod 32) words is free of bank conflicts, and the
-// U_B column of the row is held in registers.  Chunks beyond the warp's largest index are
-// skipped (warp-uniform bounds).
+// 4*VW*t + u), which with a row stride of 16 (mod 32) words is free of bank conflicts; all
+// chunk loads are issued before any FMA and every chunk has its own accumulator, so the
+// products form short independent chains.  The U_B column of the row is held in registers.
 #pragma once
 
 #include "kg_common.cuh"
+#include "kg_tc.cuh"
 
 namespace kg {
 
@@ -50,21 +51,72 @@ struct LeafSmem {
     int8_t Cs[KG_T][KG_T];
 };
 
+// Store one 16-byte vector; when a second plane is given (fp32 feeding the 3xTF32 update),
+// store the tf32 split instead: hi to dst_hi, the tf32 remainder to dst_lo.
+__device__ __forceinline__ void leaf_store_split(float* dst_hi, float* dst_lo, int64_t off, float4 v) {
+    if (dst_lo) {
+        float4 h, l;
+        tc::split_tf32(v.x, h.x, l.x);
+        tc::split_tf32(v.y, h.y, l.y);
+        tc::split_tf32(v.z, h.z, l.z);
+        tc::split_tf32(v.w, h.w, l.w);
+        *reinterpret_cast<float4*>(dst_hi + off) = h;
+        *reinterpret_cast<float4*>(dst_lo + off) = l;
+    } else {
+        *reinterpret_cast<float4*>(dst_hi + off) = v;
+    }
+}
+__device__ __forceinline__ void leaf_store_split(double* dst, double*, int64_t off, double2 v) {
+    *reinterpret_cast<double2*>(dst + off) = v;
+}
+
 template <typename Real>
 __device__ __forceinline__ Real leaf_clamp(Real v, Real lo, Real hi) {
     return v < lo ? lo : (v > hi ? hi : v);
 }
 
+// Copy a 64x64 tile of a row-major matrix (leading dimension ld) into shared memory with a
+// per-element transform, issuing all 16-byte global loads of a pass before the stores.
+template <typename Real, int PASSES, class Store>
+__device__ __forceinline__ void leaf_load_tile(const Real* __restrict__ src, int64_t ld, Store store) {
+    constexpr int VW = LeafCfg<Real>::VW;
+    constexpr int PER_ROW = KG_T / VW;                // vectors per tile row
+    constexpr int TOTAL = KG_T * PER_ROW;             // vectors per tile
+    constexpr int PER_THREAD = TOTAL / 256;           // 4 (fp32) or 8 (fp64)
+    constexpr int PER_PASS = PER_THREAD / PASSES;
+    using Vec = typename LeafCfg<Real>::V;
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+        Vec v[PER_PASS];
+#pragma unroll
+        for (int e = 0; e < PER_PASS; ++e) {
+            const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
+            const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+            v[e] = *reinterpret_cast<const Vec*>(src + (int64_t)r * ld + c);
+        }
+#pragma unroll
+        for (int e = 0; e < PER_PASS; ++e) {
+            const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
+            const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+            const Real* x = reinterpret_cast<const Real*>(&v[e]);
+#pragma unroll
+            for (int u = 0; u < VW; ++u) store(r, c + u, x[u]);
+        }
+    }
+}
+
 template <typename Real>
 __global__ void __launch_bounds__(256)
-k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
-       Real* __restrict__ Wt, Real* __restrict__ R, Real* __restrict__ Ebuf,
+k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
+       Real* __restrict__ Wt, Real* __restrict__ R, Real* __restrict__ Ebuf, Real* __restrict__ Elo,
+       Real* __restrict__ XTg, Real* __restrict__ XTlo,
        const Real* __restrict__ UA, int64_t ldA, const Real* __restrict__ UB, int64_t ldB,
        const Real* __restrict__ sp, int qmin, int qmax,
        int8_t* __restrict__ codes, Real* __restrict__ V, Real* __restrict__ outE) {
     constexpr int T = KG_T;
     constexpr int VW = LeafCfg<Real>::VW;
     constexpr int NC = T / (4 * VW);     // chunks per lane and dot product
+    constexpr int PASSES = (sizeof(Real) == 8) ? 2 : 1;
     using Vec = typename LeafCfg<Real>::V;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     LeafSmem<Real>& sm = *reinterpret_cast<LeafSmem<Real>*>(smem_raw);
@@ -76,15 +128,12 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
     // ---- load: a^T (masked), b row-major (masked) into Es, R into XT, W~ into Ws
-    for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
-        const Real av = UA[(c0 + r) * ldA + c0 + c];
-        const Real bv = UB[(r0 + r) * ldB + r0 + c];
-        sm.aT[c][r] = (c >= r) ? av : Real(0);
-        sm.Es[r][c] = (c >= r) ? bv : Real(0);
-        sm.XT[r][c] = R[(r0 + r) * Np + c0 + c];
-        sm.Ws[r][c] = Wt[(r0 + r) * Np + c0 + c];
-    }
+    leaf_load_tile<Real, PASSES>(UA + c0 * ldA + c0, ldA,
+                                 [&](int r, int c, Real x) { sm.aT[c][r] = (c >= r) ? x : Real(0); });
+    leaf_load_tile<Real, PASSES>(UB + r0 * ldB + r0, ldB,
+                                 [&](int r, int c, Real x) { sm.Es[r][c] = (c >= r) ? x : Real(0); });
+    leaf_load_tile<Real, PASSES>(R + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.XT[r][c] = x; });
+    leaf_load_tile<Real, PASSES>(Wt + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.Ws[r][c] = x; });
     if (tid < T) {
         const Real s = sp[r0 + tid];
         sm.s[tid] = s;
@@ -97,7 +146,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
     }
 
     // ---- per-row constants; U_B column of the row in registers
-    const int i = tid >> 2, q = tid & 3, w = tid >> 5;
+    const int i = tid >> 2, q = tid & 3;
     const Real b_ii = sm.Es[i][i];
     const Real b_up = (i > 0) ? sm.Es[i - 1][i] : Real(0);
     const Real invb = Real(1) / b_ii;
@@ -120,6 +169,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[a][c] = Real(0);
         const int kmax = ty * 4 + 3;
+#pragma unroll 4
         for (int k = 0; k <= kmax; ++k) {
             Real bv[4], rv[4];
 #pragma unroll
@@ -146,13 +196,42 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
 
     // ---- sweep
     const Real fqmin = Real(qmin), fqmax = Real(qmax);
-    const int imax_w = 8 * w + 7;
-    const int tc = min(NC, (imax_w - 1 + 4 * VW - 1) / (4 * VW));   // chunks with some k < i-1
     Real pre_x = Real(0), r_pre = Real(0), e_prev = Real(0), a_left = Real(0);
     Real inva_j = Real(0), ajj_j = Real(0);
+    const int w = tid >> 5;
+    // The lane's share of row i of E (k = VW*q + 4*VW*t + u) lives in registers: written by
+    // predicated moves when the row produces it, so the row-chain products read only a^T from
+    // shared memory.  Shared-memory bandwidth is what bounds a step.
+    Real ereg[NC][VW];
+#pragma unroll
+    for (int t = 0; t < NC; ++t)
+#pragma unroll
+        for (int u = 0; u < VW; ++u) ereg[t][u] = Real(0);
+    // chunks holding some k < i-1 (column chain) are fixed per warp
+    const int tc = min(NC, (8 * w + 6 + 4 * VW - 1) / (4 * VW));
     for (int d = -1; d < 2 * T - 1; ++d) {
         const int j = d - i;
+        const int jn = j + 1;
         const bool proc = (j >= 0) && (j < T);
+        const bool pre = (jn >= 0) && (jn < T);
+        const bool warp_pre = (d - 8 * w + 1 >= 0) && (d - (8 * w + 7) + 1 < T);   // warp-uniform
+        // chunks holding some k < j (row chain): the warp's largest j is d - 8w
+        const int tr = min(NC, max(0, (d - 8 * w + 4 * VW - 1) / (4 * VW)));
+        // issue the look-ahead loads first: they do not depend on this step's results
+        Vec xv[NC], av[NC];
+        Real w_next = Real(0), a_next = Real(0), inva_next = Real(0), ajj_next = Real(0);
+        if (warp_pre) {
+            const int jr = pre ? jn : 0;
+#pragma unroll
+            for (int t = 0; t < NC; ++t) {
+                if (t < tc) xv[t] = *reinterpret_cast<const Vec*>(&sm.XT[jr][VW * q + 4 * VW * t]);
+                if (t < tr) av[t] = *reinterpret_cast<const Vec*>(&sm.aT[jr][VW * q + 4 * VW * t]);
+            }
+            w_next = sm.Ws[i][jr];
+            a_next = (jr > 0) ? sm.aT[jr][jr - 1] : Real(0);
+            inva_next = sm.inva[jr];
+            ajj_next = sm.ajj[jr];
+        }
         Real e = Real(0), Q = Real(0), Xv = Real(0), code = Real(0);
         if (proc) {
             const Real x_up = (i > 0) ? sm.XT[j][i - 1] : Real(0);
@@ -163,48 +242,53 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
             e = (x - Q) * invb * inva_j;
             Xv = (r_pre + t_left) + e * ajj_j;
         }
-        // look-ahead: everything column j+1 needs except the terms produced at this step
-        const int jn = j + 1;
-        const int jmax_w = d - 8 * w;                 // largest j in the warp (row 8w)
-        if (jmax_w + 1 >= 0 && d - imax_w + 1 < T) {  // some row of the warp precomputes
-            Real c = Real(0), r = Real(0);
-            const bool pre = (jn >= 0) && (jn < T);
-            const int jr = pre ? jn : 0;
+        if (warp_pre) {
+            Real cacc[NC], racc[NC];
 #pragma unroll
             for (int t = 0; t < NC; ++t) {
+                cacc[t] = Real(0);
+                racc[t] = Real(0);
                 if (t < tc) {
-                    const Vec xv = *reinterpret_cast<const Vec*>(&sm.XT[jr][VW * q + 4 * VW * t]);
-                    const Real* xs = reinterpret_cast<const Real*>(&xv);
+                    const Real* xs = reinterpret_cast<const Real*>(&xv[t]);
 #pragma unroll
-                    for (int u = 0; u < VW; ++u) c += breg[t][u] * xs[u];
+                    for (int u = 0; u < VW; ++u) cacc[t] += breg[t][u] * xs[u];
                 }
-            }
-            const int tr = min(NC, max(0, (jmax_w + 4 * VW - 1) / (4 * VW)));   // chunks with some k < j
-#pragma unroll
-            for (int t = 0; t < NC; ++t) {
                 if (t < tr) {
-                    const Vec ev = *reinterpret_cast<const Vec*>(&sm.Es[i][VW * q + 4 * VW * t]);
-                    const Vec av = *reinterpret_cast<const Vec*>(&sm.aT[jr][VW * q + 4 * VW * t]);
-                    const Real* es = reinterpret_cast<const Real*>(&ev);
-                    const Real* as = reinterpret_cast<const Real*>(&av);
+                    const Real* as = reinterpret_cast<const Real*>(&av[t]);
 #pragma unroll
-                    for (int u = 0; u < VW; ++u) r += es[u] * as[u];
+                    for (int u = 0; u < VW; ++u) racc[t] += ereg[t][u] * as[u];
                 }
             }
+#pragma unroll
+            for (int h = NC / 2; h > 0; h >>= 1)
+#pragma unroll
+                for (int t = 0; t < h; ++t) {
+                    cacc[t] += cacc[t + h];
+                    racc[t] += racc[t + h];
+                }
+            Real c = cacc[0], r = racc[0];
             c += __shfl_xor_sync(0xffffffffu, c, 1);
-            c += __shfl_xor_sync(0xffffffffu, c, 2);
             r += __shfl_xor_sync(0xffffffffu, r, 1);
+            c += __shfl_xor_sync(0xffffffffu, c, 2);
             r += __shfl_xor_sync(0xffffffffu, r, 2);
             if (pre) {
-                // E[i][j] is still zero in shared memory here (written below), so r covers k < j
-                pre_x = sm.Ws[i][jn] - c - b_ii * r;
+                // E[i][j] enters ereg only below, so r covers k < j; b[i-1][i] is zero in breg,
+                // so c covers k < i-1
+                pre_x = w_next - c - b_ii * r;
                 r_pre = r;
-                a_left = (jn > 0) ? sm.aT[jn][jn - 1] : Real(0);
-                inva_j = sm.inva[jn];
-                ajj_j = sm.ajj[jn];
+                a_left = a_next;
+                inva_j = inva_next;
+                ajj_j = ajj_next;
             }
         }
         e_prev = e;
+        if (proc) {   // the lane owning column j keeps E[i][j]
+#pragma unroll
+            for (int t = 0; t < NC; ++t)
+#pragma unroll
+                for (int u = 0; u < VW; ++u)
+                    if (j == VW * q + 4 * VW * t + u) ereg[t][u] = e;
+        }
         __syncwarp();
         if (proc && q == 0) {
             sm.Es[i][j] = e;
@@ -215,28 +299,47 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np,
         __syncthreads();
     }
 
-    // ---- write back: codes, V, E; then the complete X = R + local X into R
-    for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
-        const int64_t gi = r0 + r, gj = c0 + c;
-        const Real ev = sm.Es[r][c];
-        Ebuf[gi * Np + gj] = ev;
-        if (gi < m && gj < n) {
-            codes[gi * n + gj] = sm.Cs[r][c];
-            V[gi * n + gj] = sm.Ws[r][c];
-            if (outE) outE[gi * n + gj] = ev;
+    // ---- write back: codes, V, E (16-byte stores where the layout allows)
+    {
+        constexpr int PER_ROW = T / VW;
+        for (int f = tid; f < T * PER_ROW; f += 256) {
+            const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+            const int64_t gi = r0 + r, gj = c0 + c;
+            Vec ev = *reinterpret_cast<const Vec*>(&sm.Es[r][c]);
+            leaf_store_split(Ebuf, Elo, gi * Np + gj, ev);
+            if (gi < m) {
+                const Real* es = reinterpret_cast<const Real*>(&ev);
+#pragma unroll
+                for (int u = 0; u < VW; ++u) {
+                    if (gj + u < n) {
+                        codes[gi * n + gj + u] = sm.Cs[r][c + u];
+                        V[gi * n + gj + u] = sm.Ws[r][c + u];
+                        if (outE) outE[gi * n + gj + u] = es[u];
+                    }
+                }
+            }
         }
     }
     __syncthreads();
+    // ---- the complete X = R + local X: back into R (row-major) and, when the tensor-core
+    //      update needs it, into XTg (X transposed, leading dimension Mp)
+    leaf_load_tile<Real, PASSES>(R + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.XT[c][r] += x; });
+    __syncthreads();
+    constexpr int PER_ROW = T / VW;
+    if (XTg) {
+        for (int f = tid; f < T * PER_ROW; f += 256) {
+            const int c = f / PER_ROW, r = (f % PER_ROW) * VW;
+            leaf_store_split(XTg, XTlo, (c0 + c) * Mp + r0 + r, *reinterpret_cast<const Vec*>(&sm.XT[c][r]));
+        }
+    }
     for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
+        const int c = idx / T, r = idx % T;
         sm.Ws[r][c] = sm.XT[c][r];
     }
     __syncthreads();
-    for (int idx = tid; idx < T * T; idx += 256) {
-        const int r = idx / T, c = idx % T;
-        const int64_t g = (r0 + r) * Np + c0 + c;
-        R[g] = R[g] + sm.Ws[r][c];
+    for (int f = tid; f < T * PER_ROW; f += 256) {
+        const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+        *reinterpret_cast<Vec*>(R + (r0 + r) * Np + c0 + c) = *reinterpret_cast<const Vec*>(&sm.Ws[r][c]);
     }
 }
 

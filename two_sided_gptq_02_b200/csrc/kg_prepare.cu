@@ -154,14 +154,13 @@ k_potrf_diag(double* __restrict__ M, int64_t kp, int kb, int64_t k, double* __re
 // L[ib,kb] = M[ib,kb] * Dinv[kb]^T for ib = kb+1 .. Kb-1 (in place; each block owns its tile)
 __global__ void __launch_bounds__(Dmma64::kThreads)
 k_panel(double* __restrict__ M, int64_t kp, int kb, const double* __restrict__ Dinv) {
-    __shared__ Dmma64::Smem sm;
+    using Pipe = DmmaPipe<false, true>;
+    __shared__ Pipe::Smem sm;
     const int ib = kb + 1 + blockIdx.x;
     double* tile = M + (int64_t)ib * NB * kp + (int64_t)kb * NB;
     Dmma64::Acc acc;
     Dmma64::zero(acc);
-    LdA_RowMajor64 la{tile, kp};
-    LdB_Trans64 lb{Dinv + (int64_t)kb * NB * NB, NB};
-    Dmma64::run(acc, sm, NB, la, lb);
+    Pipe::run(acc, sm, NB, tile, kp, Dinv + (int64_t)kb * NB * NB, NB);
     __syncthreads();
     Dmma64::for_each(acc, [&](int r, int c, double v) { tile[(int64_t)r * kp + c] = v; });
 }
@@ -169,15 +168,15 @@ k_panel(double* __restrict__ M, int64_t kp, int kb, const double* __restrict__ D
 // M[ib,jb] -= L[ib,kb] L[jb,kb]^T for kb < jb <= ib
 __global__ void __launch_bounds__(Dmma64::kThreads)
 k_syrk(double* __restrict__ M, int64_t kp, int kb) {
-    __shared__ Dmma64::Smem sm;
+    using Pipe = DmmaPipe<false, true>;
+    __shared__ Pipe::Smem sm;
     const int jb = kb + 1 + blockIdx.x;
     const int ib = kb + 1 + blockIdx.y;
     if (jb > ib) return;
     Dmma64::Acc acc;
     Dmma64::zero(acc);
-    LdA_RowMajor64 la{M + (int64_t)ib * NB * kp + (int64_t)kb * NB, kp};
-    LdB_Trans64 lb{M + (int64_t)jb * NB * kp + (int64_t)kb * NB, kp};
-    Dmma64::run(acc, sm, NB, la, lb);
+    Pipe::run(acc, sm, NB, M + (int64_t)ib * NB * kp + (int64_t)kb * NB, kp,
+              M + (int64_t)jb * NB * kp + (int64_t)kb * NB, kp);
     double* out = M + (int64_t)ib * NB * kp + (int64_t)jb * NB;
     Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] -= v; });
 }
@@ -197,13 +196,13 @@ __global__ void k_x_init(double* __restrict__ X, int64_t kp, const double* __res
 // Tmp[:, jb] = sum_{kb=jb}^{ib-1} L[ib,kb] X[kb,jb]    for jb < ib
 __global__ void __launch_bounds__(Dmma64::kThreads)
 k_inv_accum(const double* __restrict__ M, const double* __restrict__ X, int64_t kp, int ib, double* __restrict__ Tmp) {
-    __shared__ Dmma64::Smem sm;
+    using Pipe = DmmaPipe<false, false>;
+    __shared__ Pipe::Smem sm;
     const int jb = blockIdx.x;
     Dmma64::Acc acc;
     Dmma64::zero(acc);
-    LdA_RowMajor64 la{M + (int64_t)ib * NB * kp + (int64_t)jb * NB, kp};
-    LdB_RowMajor64 lb{X + (int64_t)jb * NB * kp + (int64_t)jb * NB, kp};
-    Dmma64::run(acc, sm, (ib - jb) * NB, la, lb);
+    Pipe::run(acc, sm, (ib - jb) * NB, M + (int64_t)ib * NB * kp + (int64_t)jb * NB, kp,
+              X + (int64_t)jb * NB * kp + (int64_t)jb * NB, kp);
     double* out = Tmp + (int64_t)jb * NB;
     Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] = v; });
 }
@@ -211,13 +210,12 @@ k_inv_accum(const double* __restrict__ M, const double* __restrict__ X, int64_t 
 // X[ib,jb] = -Dinv[ib] * Tmp[:, jb]
 __global__ void __launch_bounds__(Dmma64::kThreads)
 k_inv_apply(double* __restrict__ X, int64_t kp, int ib, const double* __restrict__ Dinv, const double* __restrict__ Tmp) {
-    __shared__ Dmma64::Smem sm;
+    using Pipe = DmmaPipe<false, false>;
+    __shared__ Pipe::Smem sm;
     const int jb = blockIdx.x;
     Dmma64::Acc acc;
     Dmma64::zero(acc);
-    LdA_RowMajor64 la{Dinv + (int64_t)ib * NB * NB, NB};
-    LdB_RowMajor64 lb{Tmp + (int64_t)jb * NB, kp};
-    Dmma64::run(acc, sm, NB, la, lb);
+    Pipe::run(acc, sm, NB, Dinv + (int64_t)ib * NB * NB, NB, Tmp + (int64_t)jb * NB, kp);
     double* out = X + (int64_t)ib * NB * kp + (int64_t)jb * NB;
     Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] = -v; });
 }

@@ -25,11 +25,13 @@
 //               W~[I,J] -= sum_{I': I'+J in [D0,mid)} U_B[I',I]^T X[I',J]     (column chain)
 //             Both are dense GEMMs over contiguous K ranges.
 #include <algorithm>
+#include <mutex>
 
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
 #include "kg_leaf.cuh"
 #include "kg_profile.cuh"
+#include "kg_push_tc.cuh"
 
 namespace kg {
 
@@ -46,7 +48,8 @@ struct QLayout {
     int64_t m, n, Mt, Nt, Mp, Np;
     bool padded;
     size_t es;
-    size_t off_wt, off_r, off_e, off_s, off_ua, off_ub, total;
+    size_t off_wt, off_r, off_e, off_s, off_ua, off_ub;
+    size_t off_elo, off_uat, off_uatlo, off_ubt, off_ubtlo, off_xt, off_xtlo, total;
 };
 
 static QLayout q_layout(int64_t m, int64_t n, size_t es) {
@@ -67,6 +70,19 @@ static QLayout q_layout(int64_t m, int64_t n, size_t es) {
         off = align_up(off + (size_t)(L.Mp * L.Mp) * es, 256);
     } else {
         L.off_ub = off;
+    }
+    L.off_elo = L.off_uat = L.off_uatlo = L.off_ubt = L.off_ubtlo = L.off_xt = L.off_xtlo = off;
+    if (es == 4) {
+        // the tensor-core update reads every operand K-major and pre-split into tf32 planes:
+        // E (the E buffer above holds its hi plane), U_A^T, U_B^T and X^T
+        auto plane = [&](size_t& o, int64_t elems) { o = off; off = align_up(off + (size_t)elems * es, 256); };
+        plane(L.off_elo, L.Mp * L.Np);
+        plane(L.off_uat, L.Np * L.Np);
+        plane(L.off_uatlo, L.Np * L.Np);
+        plane(L.off_ubt, L.Mp * L.Mp);
+        plane(L.off_ubtlo, L.Mp * L.Mp);
+        plane(L.off_xt, L.Np * L.Mp);
+        plane(L.off_xtlo, L.Np * L.Mp);
     }
     L.total = off;
     return L;
@@ -142,7 +158,11 @@ __global__ void __launch_bounds__(Dmma64::kThreads)
 k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
            double* __restrict__ Wt, double* __restrict__ R, const double* __restrict__ E,
            const double* __restrict__ UA, int64_t ldA, const double* __restrict__ UB, int64_t ldB) {
-    __shared__ Dmma64::Smem sm;
+    using PipeRow = DmmaPipe<false, false>;   // A = rows of E,  B = rows of U_A
+    using PipeCol = DmmaPipe<true, false>;    // A = U_B (stored K x 64), B = rows of X
+    constexpr size_t kSmem = sizeof(PipeRow::Smem) > sizeof(PipeCol::Smem) ? sizeof(PipeRow::Smem)
+                                                                            : sizeof(PipeCol::Smem);
+    __shared__ __align__(16) unsigned char smem[kSmem];
     const int D = mid + blockIdx.y;
     const int I = max(0, D - Nt + 1) + blockIdx.x;
     if (I > min(D, Mt - 1)) return;
@@ -152,17 +172,15 @@ k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
     if (blockIdx.z == 0) {
         const int k0 = max(0, D0 - I), k1 = min(Nt, mid - I);
         if (k0 >= k1) return;
-        LdA_RowMajor64 la{E + (int64_t)I * T * Np + (int64_t)k0 * T, Np};
-        LdB_RowMajor64 lb{UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA};
-        Dmma64::run(acc, sm, (k1 - k0) * T, la, lb);
+        PipeRow::run(acc, *reinterpret_cast<PipeRow::Smem*>(smem), (k1 - k0) * T,
+                     E + (int64_t)I * T * Np + (int64_t)k0 * T, Np, UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA);
         double* out = R + (int64_t)I * T * Np + (int64_t)J * T;
         Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] += v; });
     } else {
         const int k0 = max(0, D0 - J), k1 = min(Mt, mid - J);
         if (k0 >= k1) return;
-        LdA_Trans64 la{UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB};
-        LdB_RowMajor64 lb{R + (int64_t)k0 * T * Np + (int64_t)J * T, Np};
-        Dmma64::run(acc, sm, (k1 - k0) * T, la, lb);
+        PipeCol::run(acc, *reinterpret_cast<PipeCol::Smem*>(smem), (k1 - k0) * T,
+                     UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB, R + (int64_t)k0 * T * Np + (int64_t)J * T, Np);
         double* out = Wt + (int64_t)I * T * Np + (int64_t)J * T;
         Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] -= v; });
     }
@@ -210,6 +228,9 @@ struct QArgs {
     Real* V;
     Real* outE;
     cudaStream_t st;
+    DevStatus* status;
+    // split K-major operand planes of the tensor-core path (fp32 only; null otherwise)
+    Real *Elo, *XT, *XTlo, *UAT, *UATlo, *UBT, *UBTlo;
 };
 
 template <typename Real>
@@ -219,8 +240,9 @@ static int launch_leaf(const QArgs<Real>& a, int D) {
     const int ntiles = Imax - Imin + 1;
     const size_t smem = sizeof(LeafSmem<Real>);
     ProfScope ps(PK_LEAF, a.st);
-    k_leaf<Real><<<ntiles, 256, smem, a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA,
-                                              a.UB, a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
+    k_leaf<Real><<<ntiles, 256, smem, a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT,
+                                              a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V,
+                                              a.outE);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -235,9 +257,13 @@ static int launch_push(const QArgs<double>& a, int D0, int mid, int D1) {
 }
 static int launch_push(const QArgs<float>& a, int D0, int mid, int D1) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    dim3 grid(std::min(Mt, Nt), D1 - mid, 2);
+    // one CTA per pair of target tiles sharing a K range: x = row (row chain) or column
+    // (column chain), y = pair index within it, z = chain
+    dim3 grid(std::max(Mt, Nt), (D1 - mid + 1) / 2, 2);
     ProfScope ps(PK_PUSH, a.st);
-    k_push_f32<<<grid, Simt64f::kThreads, 0, a.st>>>(D0, mid, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB, a.ldB);
+    const SplitOperands op{a.E, a.Elo, a.XT, a.XTlo, a.UAT, a.UATlo, a.UBT, a.UBTlo};
+    k_push_tc32<<<grid, PushTc::THREADS, PushTc::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.L.Mp, a.Wt, a.R,
+                                                                    op, a.status);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -271,6 +297,7 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
     a.V = static_cast<Real*>(V);
     a.outE = static_cast<Real*>(outE);
     a.st = st;
+    a.status = status;
 
     KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
     const int nb = 148 * 4;
@@ -310,18 +337,49 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         a.UA = static_cast<const Real*>(UA_); a.ldA = n;
         a.UB = static_cast<const Real*>(UB_); a.ldB = m;
     }
+    a.Elo = a.XT = a.XTlo = a.UAT = a.UATlo = a.UBT = a.UBTlo = nullptr;
+    if (sizeof(Real) == 4) {
+        a.Elo = reinterpret_cast<Real*>(base + L.off_elo);
+        a.UAT = reinterpret_cast<Real*>(base + L.off_uat);
+        a.UATlo = reinterpret_cast<Real*>(base + L.off_uatlo);
+        a.UBT = reinterpret_cast<Real*>(base + L.off_ubt);
+        a.UBTlo = reinterpret_cast<Real*>(base + L.off_ubtlo);
+        a.XT = reinterpret_cast<Real*>(base + L.off_xt);
+        a.XTlo = reinterpret_cast<Real*>(base + L.off_xtlo);
+        {
+            ProfScope ps(PK_INIT, st);
+            k_transpose_split<<<nb, 256, 0, st>>>(reinterpret_cast<const float*>(a.UA), L.Np, a.ldA,
+                                                  reinterpret_cast<float*>(a.UAT), reinterpret_cast<float*>(a.UATlo));
+        }
+        KG_LAUNCH_CHECK();
+        {
+            ProfScope ps(PK_INIT, st);
+            k_transpose_split<<<nb, 256, 0, st>>>(reinterpret_cast<const float*>(a.UB), L.Mp, a.ldB,
+                                                  reinterpret_cast<float*>(a.UBT), reinterpret_cast<float*>(a.UBTlo));
+        }
+        KG_LAUNCH_CHECK();
+    }
     return solve_range(a, 0, (int)(L.Mt + L.Nt - 1));
 }
 
-static bool leaf_smem_configured[2] = {false, false};
+// Kernel attributes are per device: configure each device once (guarded by a mutex).
+static std::mutex g_cfg_mu;
+static bool g_cfg_done[2][256] = {};
 
 template <typename Real>
 static int configure_leaf() {
     const int idx = sizeof(Real) == 8 ? 1 : 0;
-    if (!leaf_smem_configured[idx]) {
+    int dev = 0;
+    KG_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 256) return KG_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_cfg_mu);
+    if (!g_cfg_done[idx][dev]) {
         KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(LeafSmem<Real>)));
-        leaf_smem_configured[idx] = true;
+        if (idx == 0)
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             PushTc::SMEM_BYTES));
+        g_cfg_done[idx][dev] = true;
     }
     return KG_OK;
 }
