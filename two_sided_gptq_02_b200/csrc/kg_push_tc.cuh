@@ -13,11 +13,14 @@
 // contiguous) from split copies the solve keeps for this purpose:
 //   row chain     A(m,k) = U_A^T[J*64+m][k],   B(k,n) = E[I*64+n][k]      D[m][n] = dR[n][m]
 //   column chain  A(m,k) = U_B^T[I*64+m][k],   B(k,n) = X^T[J*64+n][k]    D[m][n] = dW[m][n]
-// Staging is a pure copy: 16-byte cp.async granules go straight to their place in the
-// no-swizzle canonical K-major layout (core matrices of 8 rows x 16 bytes) of a 4-stage ring;
-// one thread issues the MMAs of a stage and commits them to that stage's mbarrier, which
-// gates the stage's reuse.  All waits are bounded in time and end early once another CTA of
-// the solve has recorded an error.
+// Staging is a pure copy into the 128-byte swizzled K-major layout of a 4-stage ring: a chunk
+// is 32 K-elements, so each operand row is one 128-byte line in global memory and one
+// 128-byte row in shared memory, with its 16-byte pieces permuted by the row index (mod 8).
+// Eight consecutive lanes copy one row, so every quarter-warp of a 16-byte cp.async reads a
+// whole line (one L2 request) and writes 128 distinct bytes (no bank conflict).  One thread
+// issues the MMAs of a stage and commits them to that stage's mbarrier, which gates the
+// stage's reuse.  All waits are bounded in time and end early once another CTA of the solve
+// has recorded an error.
 #pragma once
 
 #include "kg_common.cuh"
@@ -33,11 +36,8 @@ struct PushTc {
     static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;      // 48 KB
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;  // + barriers, slot, align pad
     static constexpr uint32_t TMEM_COLS = 64;
-    // K-major no-swizzle layout: core matrices (8 rows x 16 bytes) contiguous along M/N (SBO),
-    // then the 4-element K groups (LBO)
-    static constexpr uint32_t SBO = 128;
-    static constexpr uint32_t LBO_A = (M / 8) * 128;   // 2048
-    static constexpr uint32_t LBO_B = (N / 8) * 128;   // 1024
+    // 128-byte swizzled K-major layout: rows of 128 bytes, 8-row groups 1024 bytes apart
+    static constexpr uint32_t SBO = 1024;
     // about 0.1 s at 2 GHz: far beyond any legitimate wait for one stage of MMAs
     static constexpr long long MAX_WAIT_CYCLES = 200000000LL;
 };
@@ -109,9 +109,8 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
     if (!two) {
         for (int s = 0; s < S; ++s) {
             unsigned char* st = smem + s * PushTc::STAGE_BYTES;
-            for (int f = tid; f < PushTc::A_BYTES / 32; f += PushTc::THREADS) {   // upper half of each plane
-                const int kq = f / 64, rest = f % 64;                               // 64 granules per K group
-                const int off = kq * PushTc::LBO_A + 1024 + rest * 16;
+            for (int f = tid; f < PushTc::A_BYTES / 32; f += PushTc::THREADS) {   // rows 64..127 of each plane
+                const int off = PushTc::A_BYTES / 2 + f * 16;
                 *reinterpret_cast<float4*>(st + off) = make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4*>(st + PushTc::A_BYTES + off) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
@@ -130,14 +129,14 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
     auto load_chunk = [&](int c, int s) {
         unsigned char* st = smem + s * PushTc::STAGE_BYTES;
         const int64_t kb = kbase0 + (int64_t)c * PushTc::BK;
+        // granule f: row f / 8, 16-byte piece ch = f % 8 of the row's 128 bytes
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
             const int f = it * PushTc::THREADS + tid;
-            const int m8 = f & 7, kq = (f >> 3) & 7, mg = f >> 6;
-            const int mr = mg * 8 + m8;
+            const int ch = f & 7, mr = f >> 3;
             if (mr < arows) {
-                const int off = m8 * 16 + mg * PushTc::SBO + kq * PushTc::LBO_A;
-                const int64_t g = (rowA + mr) * ld + kb + 4 * kq;
+                const int off = mr * 128 + ((ch ^ (mr & 7)) << 4);
+                const int64_t g = (rowA + mr) * ld + kb + 4 * ch;
                 cp_async16(st + off, Ahi + g);
                 cp_async16(st + PushTc::A_BYTES + off, Alo + g);
             }
@@ -145,9 +144,9 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
             const int f = it * PushTc::THREADS + tid;
-            const int n8 = f & 7, kq = (f >> 3) & 7, ng = f >> 6;
-            const int off = n8 * 16 + ng * PushTc::SBO + kq * PushTc::LBO_B;
-            const int64_t g = (rowB + ng * 8 + n8) * ld + kb + 4 * kq;
+            const int ch = f & 7, nr = f >> 3;
+            const int off = nr * 128 + ((ch ^ (nr & 7)) << 4);
+            const int64_t g = (rowB + nr) * ld + kb + 4 * ch;
             cp_async16(st + 2 * PushTc::A_BYTES + off, Bhi + g);
             cp_async16(st + 2 * PushTc::A_BYTES + PushTc::B_BYTES + off, Blo + g);
         }
@@ -172,11 +171,11 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
             const uint32_t sb_hi = sa_hi + 2 * PushTc::A_BYTES, sb_lo = sb_hi + PushTc::B_BYTES;
 #pragma unroll
             for (int ks = 0; ks < PushTc::BK / 8; ++ks) {
-                // one MMA covers K = 8: two 4-element K groups
-                const uint64_t ah = tc::smem_desc(sa_hi + 2 * ks * PushTc::LBO_A, PushTc::LBO_A, PushTc::SBO);
-                const uint64_t al = tc::smem_desc(sa_lo + 2 * ks * PushTc::LBO_A, PushTc::LBO_A, PushTc::SBO);
-                const uint64_t bh = tc::smem_desc(sb_hi + 2 * ks * PushTc::LBO_B, PushTc::LBO_B, PushTc::SBO);
-                const uint64_t bl = tc::smem_desc(sb_lo + 2 * ks * PushTc::LBO_B, PushTc::LBO_B, PushTc::SBO);
+                // one MMA covers K = 8, i.e. 32 bytes of every row
+                const uint64_t ah = tc::smem_desc_sw128(sa_hi + 32 * ks, PushTc::SBO);
+                const uint64_t al = tc::smem_desc_sw128(sa_lo + 32 * ks, PushTc::SBO);
+                const uint64_t bh = tc::smem_desc_sw128(sb_hi + 32 * ks, PushTc::SBO);
+                const uint64_t bl = tc::smem_desc_sw128(sb_lo + 32 * ks, PushTc::SBO);
                 const uint32_t acc0 = (c > 0 || ks > 0) ? 1u : 0u;
                 tc::mma_tf32(tbase, al, bh, idesc, acc0);
                 tc::mma_tf32(tbase, ah, bl, idesc, 1u);

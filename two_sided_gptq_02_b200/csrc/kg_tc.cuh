@@ -46,6 +46,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     }
 }
 
+// Arrive on the barrier (release semantics at CTA scope: the caller's earlier shared-memory
+// writes are visible to whoever then sees the phase complete).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ---- TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -80,6 +86,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     d |= (uint64_t)1 << 46;   // version
     // base offset 0, lbo mode 0, layout type 0 (no swizzle)
     return d;
+}
+// Descriptor of a K-major operand in the 128-byte swizzled layout: each row's 128 bytes of K
+// are contiguous, rows follow at 128 bytes, 8-row groups at sbo bytes, and the 16-byte chunk c
+// of row r sits at chunk position c ^ (r % 8) (the swizzle acts on address bits 4-6 with bits
+// 7-9, so the operand base must be 1024-byte aligned; a K offset inside the 128 bytes is
+// applied by advancing saddr).  The leading offset is unused for this layout and set to 16.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t sbo) {
+    return smem_desc(saddr, 16u, sbo) | ((uint64_t)2 << 61);   // layout type 2: 128-byte swizzle
 }
 // Instruction descriptor for kind::tf32 with fp32 accumulation, dense.
 // a_mn / b_mn: operand stored M-(N-)major instead of K-major.
