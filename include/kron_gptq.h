@@ -48,7 +48,8 @@ typedef enum kg_status {
     KG_OK = 0,
     KG_ERR_ARG = -1,          /* null pointer, negative size, bad grid, misaligned pointer */
     KG_ERR_UNSUPPORTED = -2,  /* dtype or grid the library does not implement */
-    KG_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
+    KG_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed, or (fp32) the driver
+                                 could not encode the tensor maps of the update operands */
     KG_ERR_WORKSPACE = -4,    /* workspace smaller than *_workspace_size() */
     KG_ERR_NOT_PD = -5,       /* (device) a Cholesky pivot was not positive */
     KG_ERR_NONFINITE = -6,    /* (device) NaN/Inf in W, in the scales or in a factor diagonal */

@@ -1,27 +1,35 @@
 // kg_push_tc.cuh -- fp32 trailing band update on the 5th-generation tensor cores (tcgen05),
-// 3xTF32: every fp32 operand x is kept as two tf32 planes hi + lo (x = hi + lo to ~22 bits)
-// and each product is formed as a_hi b_hi + a_hi b_lo + a_lo b_hi, accumulated in fp32 in
-// tensor memory (TMEM).
+// 3xTF32, operands staged by the Tensor Memory Accelerator.
 //
 // The band update of "FastKron: Efficient Quantization with Kronecker-Factored Hessians",
 // Section 2.4 (W -= L^B Delta L^A^T, batched), in its two-chain form:
 //   column chain  W~[I,J] -= sum_{I'} U_B[I',I]^T X[I',J]         (I' over band 1 of column J)
 //   row chain     R[I,J]  += sum_{J'} E[I,J'] U_A[J',J]            (J' over band 1 of row I)
-// Target tiles that share a K range are paired along M: two tiles of one column (column
-// chain) or, computing R^T = U_A^T E^T, two tiles of one row (row chain).  One CTA computes
-// one 128 x 64 block with M=128, N=64, K=8 MMAs.  Both operands are read K-major (k
-// contiguous) from split copies the solve keeps for this purpose:
+// Every fp32 operand x is kept as two tf32 planes hi + lo (x = hi + lo to ~22 bits); each product
+// is a_hi b_hi + a_hi b_lo + a_lo b_hi, accumulated in fp32 in tensor memory (TMEM).
+// Target tiles that share a K range are paired along M: two tiles of one column (column chain)
+// or, computing R^T = U_A^T E^T, two tiles of one row (row chain).  One CTA computes one 128 x 64
+// block with M=128, N=64, K=8 MMAs.  Both operands are read K-major (k contiguous) from split
+// copies the solve keeps for this purpose:
 //   row chain     A(m,k) = U_A^T[J*64+m][k],   B(k,n) = E[I*64+n][k]      D[m][n] = dR[n][m]
 //   column chain  A(m,k) = U_B^T[I*64+m][k],   B(k,n) = X^T[J*64+n][k]    D[m][n] = dW[m][n]
-// Staging is a pure copy into the 128-byte swizzled K-major layout of a 4-stage ring: a chunk
-// is 32 K-elements, so each operand row is one 128-byte line in global memory and one
-// 128-byte row in shared memory, with its 16-byte pieces permuted by the row index (mod 8).
-// Eight consecutive lanes copy one row, so every quarter-warp of a 16-byte cp.async reads a
-// whole line (one L2 request) and writes 128 distinct bytes (no bank conflict).  One thread
-// issues the MMAs of a stage and commits them to that stage's mbarrier, which gates the
-// stage's reuse.  All waits are bounded in time and end early once another CTA of the solve
-// has recorded an error.
+// Staging: a chunk is 32 K-elements, so each operand row is one 128-byte line; tensor-map loads
+// of 64-row x 32-element boxes land in the 128-byte swizzled K-major layout the MMA descriptors
+// name (16-byte pieces of row r permuted by r mod 8).  In a CTA of four warps
+//   * one producer thread (warp 0) issues the loads of a stage, completing on the stage's "full"
+//     mbarrier by transaction count;
+//   * one MMA thread (warp 1) waits for a full stage, issues its 12 MMAs and commits them to
+//     the stage's "empty" mbarrier, which the producer waits on before refilling it (4 stages);
+//   * all four warps meet only at the end, to drain the accumulator from TMEM.
+// Every wait is bounded in time and ends early once the solve has recorded an error; before the
+// CTA exits it waits (bounded, without early exit) for the loads it issued and the MMAs it
+// committed.
 #pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
@@ -31,10 +39,13 @@ namespace kg {
 
 struct PushTc {
     static constexpr int M = 128, N = 64, BK = 32, STAGES = 4, THREADS = 128;
+    // one chunk = BK = 32 K-elements = one 128-byte line per operand row
     static constexpr int A_BYTES = M * BK * 4;                         // 16 KB per plane
     static constexpr int B_BYTES = N * BK * 4;                         //  8 KB
     static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;      // 48 KB
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;  // + barriers, slot, align pad
+    static constexpr int BOX_BYTES = 64 * BK * 4;                      // one 64-row box of one plane
+    // + barriers (full[S], empty[S], done), TMEM slot, counters; + pad to a 1024-byte base
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
     static constexpr uint32_t TMEM_COLS = 64;
     // 128-byte swizzled K-major layout: rows of 128 bytes, 8-row groups 1024 bytes apart
     static constexpr uint32_t SBO = 1024;
@@ -48,17 +59,42 @@ struct SplitOperands {
     const float *E_hi, *E_lo, *XT_hi, *XT_lo, *UAT_hi, *UAT_lo, *UBT_hi, *UBT_lo;
 };
 
-__global__ void __launch_bounds__(PushTc::THREADS)
-k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, float* __restrict__ Wt,
-            float* __restrict__ R, SplitOperands op, DevStatus* status) {
+// Tensor maps of the eight split planes (2-D, inner dimension = K, box 32 x 64, 128-byte
+// swizzle).  E* are Mp x Np, XT* Np x Mp, UAT* Np x Np, UBT* Mp x Mp (rows x inner).
+struct PushTmaMaps {
+    CUtensorMap E_hi, E_lo, XT_hi, XT_lo, UAT_hi, UAT_lo, UBT_hi, UBT_lo;
+};
+
+namespace tc {
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// 2-D tiled bulk tensor load global -> shared, completing on bar; x = inner (K) coordinate in
+// elements (a multiple of 32 here, so 16-byte aligned), y = row coordinate
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+}  // namespace tc
+
+__global__ void __launch_bounds__(PushTc::THREADS, 1)
+k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restrict__ Wt, float* __restrict__ R,
+            const __grid_constant__ PushTmaMaps maps, DevStatus* status) {
     constexpr int T = KG_T;
     constexpr int S = PushTc::STAGES;
     extern __shared__ __align__(16) unsigned char smem_tc_raw[];
-    // 1024-byte aligned base for the operand stages (the launch reserves the padding)
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_tc_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + S * PushTc::STAGE_BYTES);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S * PushTc::STAGE_BYTES + 128);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * PushTc::STAGE_BYTES);
+    uint64_t* empty = full + S;
+    uint64_t* done = empty + S;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+    int* issued_s = reinterpret_cast<int*>(tslot + 1);     // chunks whose loads were issued
+    int* consumed_s = issued_s + 1;                         // chunks whose MMAs were issued
 
     const int chain = blockIdx.z;   // 0: row chain (into R), 1: column chain (into W~)
     int I, J, k0, k1;
@@ -86,35 +122,38 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
     // a solve that already failed (time-out, bad input) does no further tensor-core work
     if (*reinterpret_cast<const volatile int*>(&status->code) != 0) return;
     const int nchunks = (k1 - k0) * (T / PushTc::BK);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // K-major operand rows: A rows start at rowA (128, or 64 when the pair is a single tile),
-    // B rows at rowB (64)
-    const float* Ahi = (chain == 1) ? op.UBT_hi : op.UAT_hi;
-    const float* Alo = (chain == 1) ? op.UBT_lo : op.UAT_lo;
-    const float* Bhi = (chain == 1) ? op.XT_hi : op.E_hi;
-    const float* Blo = (chain == 1) ? op.XT_lo : op.E_lo;
-    const int64_t ld = (chain == 1) ? Mp : Np;
-    const int64_t rowA = (chain == 1) ? (int64_t)I * T : (int64_t)J * T;
-    const int64_t rowB = (chain == 1) ? (int64_t)J * T : (int64_t)I * T;
-    const int64_t kbase0 = (int64_t)k0 * T;
-    const int arows = two ? 128 : 64;
+    const CUtensorMap* mAh = (chain == 1) ? &maps.UBT_hi : &maps.UAT_hi;
+    const CUtensorMap* mAl = (chain == 1) ? &maps.UBT_lo : &maps.UAT_lo;
+    const CUtensorMap* mBh = (chain == 1) ? &maps.XT_hi : &maps.E_hi;
+    const CUtensorMap* mBl = (chain == 1) ? &maps.XT_lo : &maps.E_lo;
+    const int rowA = (chain == 1) ? I * T : J * T;
+    const int rowB = (chain == 1) ? J * T : I * T;
+    const uint32_t chunk_bytes = (uint32_t)((two ? 4 : 2) + 2) * PushTc::BOX_BYTES;
 
     if (tid == 0) {
 #pragma unroll
-        for (int s = 0; s < S; ++s) tc::mbar_init(&mbar[s], 1);
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(done, 1);
+        *issued_s = 0;
+        *consumed_s = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // rows of A beyond a single tile stay zero in every stage
+    // rows 64..127 of A stay zero in every stage when the pair is a single tile
     if (!two) {
         for (int s = 0; s < S; ++s) {
             unsigned char* st = smem + s * PushTc::STAGE_BYTES;
-            for (int f = tid; f < PushTc::A_BYTES / 32; f += PushTc::THREADS) {   // rows 64..127 of each plane
+            for (int f = tid; f < PushTc::A_BYTES / 32; f += PushTc::THREADS) {
                 const int off = PushTc::A_BYTES / 2 + f * 16;
                 *reinterpret_cast<float4*>(st + off) = make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4*>(st + PushTc::A_BYTES + off) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
+        tc::fence_proxy_async_smem();
     }
     if (warp == 0) {
         tc::tmem_alloc(tslot, PushTc::TMEM_COLS);
@@ -124,54 +163,45 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tslot;
+    bool ok = true;
 
-    // copy of chunk c into stage s: A = arows x 32, B = 64 x 32, both planes
-    auto load_chunk = [&](int c, int s) {
-        unsigned char* st = smem + s * PushTc::STAGE_BYTES;
-        const int64_t kb = kbase0 + (int64_t)c * PushTc::BK;
-        // granule f: row f / 8, 16-byte piece ch = f % 8 of the row's 128 bytes
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int f = it * PushTc::THREADS + tid;
-            const int ch = f & 7, mr = f >> 3;
-            if (mr < arows) {
-                const int off = mr * 128 + ((ch ^ (mr & 7)) << 4);
-                const int64_t g = (rowA + mr) * ld + kb + 4 * ch;
-                cp_async16(st + off, Ahi + g);
-                cp_async16(st + PushTc::A_BYTES + off, Alo + g);
+    if (warp == 0 && lane == 0) {
+        // ---- producer
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % S;
+            if (c >= S && !tc::mbar_wait(&empty[s], (uint32_t)(((c / S) - 1) & 1), PushTc::MAX_WAIT_CYCLES,
+                                         &status->code)) {
+                ok = false;
+                break;
             }
+            unsigned char* st = smem + s * PushTc::STAGE_BYTES;
+            const int kx = (k0 * T) + c * PushTc::BK;
+            tc::mbar_arrive_expect_tx(&full[s], chunk_bytes);
+            tc::tma_load_2d(st, mAh, kx, rowA, &full[s]);
+            tc::tma_load_2d(st + PushTc::A_BYTES, mAl, kx, rowA, &full[s]);
+            if (two) {
+                tc::tma_load_2d(st + PushTc::BOX_BYTES, mAh, kx, rowA + T, &full[s]);
+                tc::tma_load_2d(st + PushTc::A_BYTES + PushTc::BOX_BYTES, mAl, kx, rowA + T, &full[s]);
+            }
+            tc::tma_load_2d(st + 2 * PushTc::A_BYTES, mBh, kx, rowB, &full[s]);
+            tc::tma_load_2d(st + 2 * PushTc::A_BYTES + PushTc::B_BYTES, mBl, kx, rowB, &full[s]);
+            *reinterpret_cast<volatile int*>(issued_s) = c + 1;
         }
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int f = it * PushTc::THREADS + tid;
-            const int ch = f & 7, nr = f >> 3;
-            const int off = nr * 128 + ((ch ^ (nr & 7)) << 4);
-            const int64_t g = (rowB + nr) * ld + kb + 4 * ch;
-            cp_async16(st + 2 * PushTc::A_BYTES + off, Bhi + g);
-            cp_async16(st + 2 * PushTc::A_BYTES + PushTc::B_BYTES + off, Blo + g);
-        }
-    };
-
-    const uint32_t idesc = tc::idesc_tf32(PushTc::M, PushTc::N, false, false);
-#pragma unroll
-    for (int s = 0; s < S - 1; ++s) {
-        if (s < nchunks) load_chunk(s, s);
-        cp_async_commit();
-    }
-    int issued = 0;   // chunks whose MMAs have been issued and committed
-    for (int c = 0; c < nchunks; ++c) {
-        const int s = c % S;
-        cp_async_wait<S - 2>();          // this thread's copies of chunk c have landed
-        tc::fence_proxy_async_smem();    // ... and are visible to the tensor core
-        __syncthreads();
-        if (tid == 0) {
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer
+        const uint32_t idesc = tc::idesc_tf32(PushTc::M, PushTc::N, false, false);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % S;
+            if (!tc::mbar_wait(&full[s], (uint32_t)((c / S) & 1), PushTc::MAX_WAIT_CYCLES, &status->code)) {
+                ok = false;
+                break;
+            }
             tc::fence_after_sync();
             unsigned char* st = smem + s * PushTc::STAGE_BYTES;
             const uint32_t sa_hi = tc::smem_u32(st), sa_lo = sa_hi + PushTc::A_BYTES;
             const uint32_t sb_hi = sa_hi + 2 * PushTc::A_BYTES, sb_lo = sb_hi + PushTc::B_BYTES;
 #pragma unroll
             for (int ks = 0; ks < PushTc::BK / 8; ++ks) {
-                // one MMA covers K = 8, i.e. 32 bytes of every row
                 const uint64_t ah = tc::smem_desc_sw128(sa_hi + 32 * ks, PushTc::SBO);
                 const uint64_t al = tc::smem_desc_sw128(sa_lo + 32 * ks, PushTc::SBO);
                 const uint64_t bh = tc::smem_desc_sw128(sb_hi + 32 * ks, PushTc::SBO);
@@ -181,31 +211,29 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
                 tc::mma_tf32(tbase, ah, bl, idesc, 1u);
                 tc::mma_tf32(tbase, ah, bh, idesc, 1u);
             }
-            tc::mma_commit(&mbar[s]);
+            tc::mma_commit(&empty[s]);
+            *reinterpret_cast<volatile int*>(consumed_s) = c + 1;
         }
-        issued = c + 1;
-        // refill the stage chunk c-1 used, once its MMAs are done
-        const int cn = c + S - 1;
-        if (cn < nchunks) {
-            bool freed = true;
-            if (c >= 1) freed = tc::mbar_wait(&mbar[(c - 1) % S], ((c - 1) / S) & 1, PushTc::MAX_WAIT_CYCLES,
-                                              &status->code);
-            if (!__syncthreads_and(freed)) break;
-            load_chunk(cn, cn % S);
-        }
-        cp_async_commit();
+        // completes once every MMA this thread issued has finished
+        tc::mma_commit(done);
     }
-    cp_async_wait<0>();
-    // ---- wait for the last issued commit (it covers every earlier MMA of this thread)
-    bool done = true;
-    if (issued > 0)
-        done = tc::mbar_wait(&mbar[(issued - 1) % S], ((issued - 1) / S) & 1, PushTc::MAX_WAIT_CYCLES,
-                             &status->code);
-    done = __syncthreads_and(done) && issued == nchunks;
-    if (!done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
+    if (!ok) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
+    __syncthreads();
+    // ---- drain: the MMAs (done) and any loads issued but never consumed, without early exit
+    const int never = 0;
+    bool drained = tc::mbar_wait(done, 0u, PushTc::MAX_WAIT_CYCLES, &never);
+    if (warp == 0 && lane == 0) {
+        const int consumed = *reinterpret_cast<volatile int*>(consumed_s);
+        const int issued = *reinterpret_cast<volatile int*>(issued_s);
+        for (int c = consumed; c < issued; ++c)
+            drained &= tc::mbar_wait(&full[c % S], (uint32_t)((c / S) & 1), PushTc::MAX_WAIT_CYCLES, &never);
+    }
+    const bool all_done = __syncthreads_and(drained) &&
+                          *reinterpret_cast<volatile int*>(consumed_s) == nchunks;
+    if (!all_done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
     tc::fence_after_sync();
-    if (done) {
-        const int mrow = warp * 32 + (tid & 31);
+    if (all_done) {
+        const int mrow = warp * 32 + lane;
         const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
         const bool valid = two || mrow < 64;
 #pragma unroll
@@ -237,6 +265,44 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, int64_t Mp, flo
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tbase, PushTc::TMEM_COLS);
+}
+
+// ---- host: tensor maps.  cuTensorMapEncodeTiled is a driver entry point; it is looked up once
+// through the runtime so the library needs no link-time dependency on libcuda.
+static PFN_cuTensorMapEncodeTiled_v12000 push_tma_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a row-major rows x inner fp32 matrix: box 32 (inner) x 64 (rows), 128-byte
+// swizzle, zero fill outside.  The base must be 16-byte aligned and inner a multiple of 4.
+static bool push_tma_map(CUtensorMap* map, const float* base, int64_t inner, int64_t rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = push_tma_encoder();
+    if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (inner & 3) != 0) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)inner * sizeof(float)};
+    const cuuint32_t box[2] = {(cuuint32_t)PushTc::BK, 64u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Maps of the eight planes; Np, Mp are the padded layer sizes (multiples of 64).
+static bool push_tma_maps(PushTmaMaps* mp, const SplitOperands& op, int64_t Np, int64_t Mp) {
+    return push_tma_map(&mp->E_hi, op.E_hi, Np, Mp) && push_tma_map(&mp->E_lo, op.E_lo, Np, Mp) &&
+           push_tma_map(&mp->XT_hi, op.XT_hi, Mp, Np) && push_tma_map(&mp->XT_lo, op.XT_lo, Mp, Np) &&
+           push_tma_map(&mp->UAT_hi, op.UAT_hi, Np, Np) && push_tma_map(&mp->UAT_lo, op.UAT_lo, Np, Np) &&
+           push_tma_map(&mp->UBT_hi, op.UBT_hi, Mp, Mp) && push_tma_map(&mp->UBT_lo, op.UBT_lo, Mp, Mp);
 }
 
 // U^T split into tf32 planes: UT_hi[c][r] + UT_lo[c][r] = U[r][c] (k x k, k multiple of 32)

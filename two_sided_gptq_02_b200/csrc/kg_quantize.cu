@@ -231,6 +231,8 @@ struct QArgs {
     DevStatus* status;
     // split K-major operand planes of the tensor-core path (fp32 only; null otherwise)
     Real *Elo, *XT, *XTlo, *UAT, *UATlo, *UBT, *UBTlo;
+    // their tensor maps (fp32 only)
+    const PushTmaMaps* maps;
 };
 
 template <typename Real>
@@ -261,9 +263,8 @@ static int launch_push(const QArgs<float>& a, int D0, int mid, int D1) {
     // (column chain), y = pair index within it, z = chain
     dim3 grid(std::max(Mt, Nt), (D1 - mid + 1) / 2, 2);
     ProfScope ps(PK_PUSH, a.st);
-    const SplitOperands op{a.E, a.Elo, a.XT, a.XTlo, a.UAT, a.UATlo, a.UBT, a.UBTlo};
-    k_push_tc32<<<grid, PushTc::THREADS, PushTc::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.L.Mp, a.Wt, a.R,
-                                                                    op, a.status);
+    k_push_tc32<<<grid, PushTc::THREADS, PushTc::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt, a.R,
+                                                                      *a.maps, a.status);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -338,6 +339,8 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         a.UB = static_cast<const Real*>(UB_); a.ldB = m;
     }
     a.Elo = a.XT = a.XTlo = a.UAT = a.UATlo = a.UBT = a.UBTlo = nullptr;
+    a.maps = nullptr;
+    PushTmaMaps maps;
     if (sizeof(Real) == 4) {
         a.Elo = reinterpret_cast<Real*>(base + L.off_elo);
         a.UAT = reinterpret_cast<Real*>(base + L.off_uat);
@@ -346,6 +349,12 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         a.UBTlo = reinterpret_cast<Real*>(base + L.off_ubtlo);
         a.XT = reinterpret_cast<Real*>(base + L.off_xt);
         a.XTlo = reinterpret_cast<Real*>(base + L.off_xtlo);
+        const SplitOperands op{reinterpret_cast<const float*>(a.E), reinterpret_cast<const float*>(a.Elo),
+                               reinterpret_cast<const float*>(a.XT), reinterpret_cast<const float*>(a.XTlo),
+                               reinterpret_cast<const float*>(a.UAT), reinterpret_cast<const float*>(a.UATlo),
+                               reinterpret_cast<const float*>(a.UBT), reinterpret_cast<const float*>(a.UBTlo)};
+        if (!push_tma_maps(&maps, op, L.Np, L.Mp)) return KG_ERR_CUDA;
+        a.maps = &maps;
         {
             ProfScope ps(PK_INIT, st);
             k_transpose_split<<<nb, 256, 0, st>>>(reinterpret_cast<const float*>(a.UA), L.Np, a.ldA,
@@ -374,11 +383,22 @@ static int configure_leaf() {
     if (dev < 0 || dev >= 256) return KG_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_cfg_mu);
     if (!g_cfg_done[idx][dev]) {
+        // The solve alternates leaf and update launches.  All of them ask for the largest
+        // shared-memory carveout, so the SMs never switch their L1 / shared split between two
+        // launches of one solve.
         KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(LeafSmem<Real>)));
-        if (idx == 0)
+        KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared));
+        if (idx == 0) {
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              PushTc::SMEM_BYTES));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
+        } else {
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_f64, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
+        }
         g_cfg_done[idx][dev] = true;
     }
     return KG_OK;
