@@ -3,13 +3,13 @@
 //
 //   Dmma64  : fp64, 128 threads (4 warps, 2x2 warp tiles of 32x32), mma.sync m8n8k4 f64
 //             (the FP64 tensor path of sm_100a; tcgen05 has no f64 kind).
-//   Simt64f : fp32, 256 threads, 4x4 outputs per thread, fp32 FMA.
 //
-// Both engines take loader functors so that each caller decides where the operands come
-// from (row-major, transposed, converted, computed on the fly):
-//   la(k0, As) fills As[r][kk] = A(r, k0+kk)   (Dmma64)      As[kk][r] (Simt64f)
+// Dmma64 takes loader functors so that each caller decides where the operands come from
+// (row-major, transposed, computed on the fly):
+//   la(k0, As) fills As[r][kk] = A(r, k0+kk)
 //   lb(k0, Bs) fills Bs[kk][c] = B(k0+kk, c)
-// and accumulate acc += A(0:64, 0:K) * B(0:K, 0:64).  K must be a multiple of BK.
+// and accumulates acc += A(0:64, 0:K) * B(0:K, 0:64).  K must be a multiple of BK.
+// DmmaPipe is the same arithmetic with cp.async double-buffered staging of plain copies.
 #pragma once
 
 #include "kg_common.cuh"
@@ -80,6 +80,31 @@ struct Dmma64 {
                 const int c = wn + ni * 8 + 2 * (lane & 3);
                 f(r, c, acc.c[mi][ni][0]);
                 f(r, c + 1, acc.c[mi][ni][1]);
+            }
+    }
+    // out[r][c] += sign * acc[r][c] on a 64 x 64 tile (row-major, leading dimension ld, 16-byte
+    // aligned rows).  All loads are issued before any store: one memory round trip in total.
+    __device__ static __forceinline__ void add_to(const Acc& acc, double* out, int64_t ld, double sign) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+        double2 o[4][4];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni) {
+                const int r = wm + mi * 8 + (lane >> 2);
+                const int c = wn + ni * 8 + 2 * (lane & 3);
+                o[mi][ni] = *reinterpret_cast<const double2*>(out + (int64_t)r * ld + c);
+            }
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni) {
+                const int r = wm + mi * 8 + (lane >> 2);
+                const int c = wn + ni * 8 + 2 * (lane & 3);
+                o[mi][ni].x += sign * acc.c[mi][ni][0];
+                o[mi][ni].y += sign * acc.c[mi][ni][1];
+                *reinterpret_cast<double2*>(out + (int64_t)r * ld + c) = o[mi][ni];
             }
     }
 };
@@ -230,86 +255,6 @@ struct DmmaPipe {
                     for (int ni = 0; ni < 4; ++ni) Dmma64::mma(acc.c[mi][ni][0], acc.c[mi][ni][1], a[mi], b[ni]);
             }
             __syncthreads();
-        }
-    }
-};
-
-// ------------------------------------------------------------------------------ fp32
-struct Simt64f {
-    static constexpr int BM = 64, BN = 64, BK = 32;
-    static constexpr int S = 64 + 4;
-    static constexpr int kThreads = 256;
-    struct Smem {
-        float As[BK][S];   // k-major
-        float Bs[BK][S];
-    };
-    struct Acc {
-        float c[4][4];
-    };
-    __device__ static __forceinline__ void zero(Acc& a) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a.c[i][j] = 0.f;
-    }
-    template <class LA, class LB>
-    __device__ static __forceinline__ void run(Acc& acc, Smem& sm, int K, LA la, LB lb) {
-        const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-        for (int k0 = 0; k0 < K; k0 += BK) {
-            __syncthreads();
-            la(k0, sm.As);
-            lb(k0, sm.Bs);
-            __syncthreads();
-#pragma unroll 8
-            for (int kk = 0; kk < BK; ++kk) {
-                const float4 a = *reinterpret_cast<const float4*>(&sm.As[kk][ty * 4]);
-                const float4 b = *reinterpret_cast<const float4*>(&sm.Bs[kk][tx * 4]);
-                const float av[4] = {a.x, a.y, a.z, a.w};
-                const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc.c[i][j] = fmaf(av[i], bv[j], acc.c[i][j]);
-            }
-        }
-    }
-    template <class F>
-    __device__ static __forceinline__ void for_each(const Acc& acc, F f) {
-        const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) f(ty * 4 + i, tx * 4 + j, acc.c[i][j]);
-    }
-};
-
-// A(r,k) = src[r * ld + k0 + k] stored k-major into As[k][r]
-struct LdAf_RowMajor {
-    const float* src; int64_t ld;
-    __device__ void operator()(int k0, float (*As)[Simt64f::S]) const {
-        for (int idx = threadIdx.x; idx < 64 * Simt64f::BK; idx += Simt64f::kThreads) {
-            const int r = idx / Simt64f::BK, k = idx % Simt64f::BK;
-            As[k][r] = src[(int64_t)r * ld + k0 + k];
-        }
-    }
-};
-// A(r,k) = src[(k0 + k) * ld + r]
-struct LdAf_Trans {
-    const float* src; int64_t ld;
-    __device__ void operator()(int k0, float (*As)[Simt64f::S]) const {
-        for (int idx = threadIdx.x; idx < 64 * Simt64f::BK; idx += Simt64f::kThreads) {
-            const int k = idx / 64, r = idx % 64;
-            As[k][r] = src[(int64_t)(k0 + k) * ld + r];
-        }
-    }
-};
-// B(k,c) = src[(k0 + k) * ld + c]
-struct LdBf_RowMajor {
-    const float* src; int64_t ld;
-    __device__ void operator()(int k0, float (*Bs)[Simt64f::S]) const {
-        for (int idx = threadIdx.x; idx < 64 * Simt64f::BK; idx += Simt64f::kThreads) {
-            const int k = idx / 64, c = idx % 64;
-            Bs[k][c] = src[(int64_t)(k0 + k) * ld + c];
         }
     }
 };

@@ -1,0 +1,396 @@
+// kg_leaf_ws.cuh -- the fp32 in-tile sweep ("leaf") with warp specialisation.
+//
+// Same in-tile problem as k_leaf in kg_leaf.cuh ("FastKron: Efficient Quantization with
+// Kronecker-Factored Hessians", Sections 2.3-2.4, restated on one tile with a = U_A[J,J],
+// b = U_B[I,I]):
+//     w'   = W~[I,J] - b^T R[I,J]
+//     r_ij = sum_{k<j} E_ik a[k][j],   c_ij = sum_{k<i} b[k][i] X_kj,   X_kj = r_kj + E_kj a[j][j]
+//     x    = w'_ij - c_ij - b_ii r_ij,  code = clamp(rint(x / s_i)),  Q = s_i code,
+//     E_ij = (x - Q) / (b_ii a_jj)
+// and the same outputs, but the 127 steps of the sweep are split between roles:
+//   * the rounding warp (warp 16) owns rows 2l and 2l+1 in lane l.  For entry (i, j) at step d
+//     it takes the helpers' partial sums
+//         P  = w'_ij - sum_{k<=i-4} b[k][i] X[k][j],     r' = sum_{k<=j-4} E[i][k] a[k][j]
+//     and adds the six newest terms itself: X of rows i-1..i-3 in column j and E of row i in
+//     columns j-1..j-3 (made at steps d-1..d-3; X of row i-1 is the lane's own other row or one
+//     shuffle away).  Only the terms of step d-1 are on its dependent chain.  It publishes E, X
+//     and the code of every entry to shared memory.
+//   * two groups of eight helper warps (four threads per row) alternate steps: the group of step
+//     d starts as soon as step d-4 is published, so each group has two rounding steps to deliver
+//     (P, r') into an eight-slot ring.  A helper thread reads one column of X, one column of a and
+//     one row of E in 16-byte chunks (k = 4q + 16t + u, lanes of a quad interleaved; row stride 16
+//     (mod 32) words, so no bank conflicts) and multiplies with packed fp32x2 FMAs; the row's
+//     U_B column stays in registers.  Reads of entries published concurrently meet a zero
+//     coefficient (b and a are masked to k <= i-4 and k <= j-4), so they cannot change a sum.
+// Hand-off goes through mbarriers, one per ring slot: arrival releases the writer's shared-memory
+// stores, a waiting warp sleeps in try_wait, every wait is bounded in time, and on expiry the CTA
+// records a time-out and skips the rest.  No slot is reused before its previous phase was seen by
+// every waiter: the rounding warp cannot finish step d+8 before both helper groups finished step
+// d+5, and a helper cannot start step d+8 before step d+4 is published.
+#pragma once
+
+#include "kg_common.cuh"
+#include "kg_leaf.cuh"
+#include "kg_tc.cuh"
+
+namespace kg {
+
+constexpr int WS_AHEAD = 4;                                  // helpers run this many steps ahead
+constexpr int WS_RING = 8;                                   // slots of the (P, r') ring
+constexpr int WS_GROUPS = 2;                                 // helper groups, alternating steps
+constexpr int WS_HELPERS = 256 * WS_GROUPS;                  // eight warps per group
+constexpr int WS_THREADS = WS_HELPERS + 32;                  // + the rounding warp
+constexpr long long WS_MAX_WAIT_CYCLES = 50000000LL;         // ~25 ms: far beyond any hand-off
+
+struct LeafWsSmem {
+    static constexpr int S = LeafCfg<float>::S;
+    float aT[KG_T][S];             // aT[j][k] = a[k][j] for k <= j - 4, else 0
+    float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
+    float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
+    float Ws[KG_T][S];             // w'
+    float colc[KG_T][8];           // column j: a[j-1][j], a[j-2][j], a[j-3][j], 1/a[j][j], a[j][j]
+    float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
+    float s[KG_T], invs[KG_T];
+    int8_t Cs[KG_T][KG_T];
+    uint64_t cbar[WS_RING];        // step d published (32 arrivals)
+    uint64_t hbar[WS_RING];        // (P, r') of step d written (one arrival per row)
+    int abort_flag;
+};
+
+// partial dots of one helper lane: c = sum breg * xv, r = sum ev * av over its 16 k
+__device__ __forceinline__ void ws_dots(const float (&breg)[4][4], const float4 (&xv)[4], const float4 (&av)[4],
+                                        const float4 (&ev)[4], float& c, float& r) {
+    float2 c0 = make_float2(0.f, 0.f), c1 = c0, r0 = c0, r1 = c0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        c0 = __ffma2_rn(make_float2(breg[t][0], breg[t][1]), make_float2(xv[t].x, xv[t].y), c0);
+        c1 = __ffma2_rn(make_float2(breg[t][2], breg[t][3]), make_float2(xv[t].z, xv[t].w), c1);
+        r0 = __ffma2_rn(make_float2(ev[t].x, ev[t].y), make_float2(av[t].x, av[t].y), r0);
+        r1 = __ffma2_rn(make_float2(ev[t].z, ev[t].w), make_float2(av[t].z, av[t].w), r1);
+    }
+    c = (c0.x + c0.y) + (c1.x + c1.y);
+    r = (r0.x + r0.y) + (r1.x + r1.y);
+}
+
+// column constants of j: a1, a2, a3, 1/ajj, ajj
+__device__ __forceinline__ void ws_ldcol(const float* p, float (&o)[5]) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
+    o[4] = p[4];
+}
+
+// The rounding warp: lane l owns rows 2l (r = 0) and 2l+1 (r = 1).
+__device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)[2], const float (&b1)[2],
+                                              const float (&b2)[2], const float (&b3)[2], const float (&sr)[2],
+                                              const float (&isr)[2], const float (&ib)[2], float fqmin, float fqmax) {
+    constexpr int T = KG_T;
+    const int l = threadIdx.x & 31;
+    float cpre[4], npre[4], ccol[2][5], ncol[2][5];
+    auto load_step = [&](int d, float (&pre)[4], float (&col)[2][5]) {
+        const float4 p = *reinterpret_cast<const float4*>(&sm.pre[d % WS_RING][2 * l][0]);
+        pre[0] = p.x; pre[1] = p.y; pre[2] = p.z; pre[3] = p.w;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int j = d - 2 * l - r;
+            ws_ldcol(&sm.colc[(unsigned)j < (unsigned)T ? j : 0][0], col[r]);
+        }
+    };
+    if (!tc::mbar_wait(&sm.hbar[0], 0u, WS_MAX_WAIT_CYCLES, &sm.abort_flag)) return false;
+    load_step(0, cpre, ccol);
+    float e1[2] = {0.f, 0.f}, e2[2] = {0.f, 0.f}, e3[2] = {0.f, 0.f};   // own E, 1..3 steps ago
+    float uo1_1 = 0.f, uo1_2 = 0.f;               // shfl_up(X_odd, 1): X of row 2l-1, 1 and 2 steps ago
+    float ue1_1 = 0.f, ue1_2 = 0.f, ue1_3 = 0.f;  // shfl_up(X_even, 1): X of row 2l-2, 1..3 steps ago
+    float uo2_1 = 0.f, uo2_2 = 0.f, uo2_3 = 0.f;  // shfl_up(X_odd, 2): X of row 2l-3, 1..3 steps ago
+    float xe_1 = 0.f;                             // own X of row 2l, 1 step ago
+    for (int d = 0; d < 2 * T - 1; ++d) {
+        // prefetch the next step's inputs; the helpers are normally ahead
+        if (d + 1 < 2 * T - 1) {
+            if (!tc::mbar_wait(&sm.hbar[(d + 1) % WS_RING], (uint32_t)(((d + 1) / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
+                               &sm.abort_flag))
+                return false;
+            load_step(d + 1, npre, ncol);
+        }
+        float e[2], X[2], code[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float xm1 = r ? xe_1 : uo1_1;    // X[i-1][j]
+            const float xm2 = r ? uo1_2 : ue1_2;   // X[i-2][j]
+            const float xm3 = r ? ue1_3 : uo2_3;   // X[i-3][j]
+            const float P = cpre[2 * r], rh = cpre[2 * r + 1];
+            // terms known before this step's chain starts
+            const float rp = (rh + e3[r] * ccol[r][2]) + e2[r] * ccol[r][1];
+            const float base = ((P - b3[r] * xm3) - b2[r] * xm2) - bii[r] * rp;
+            // the chain: E[i][j-1] and X[i-1][j] were made at step d-1
+            const float t1 = e1[r] * ccol[r][0];
+            const float x = (base - bii[r] * t1) - b1[r] * xm1;
+            code[r] = leaf_clamp(rintf(x * isr[r]), fqmin, fqmax);
+            const float Q = code[r] * sr[r];
+            e[r] = (x - Q) * (ib[r] * ccol[r][3]);
+            X[r] = (rp + t1) + e[r] * ccol[r][4];
+            const int j = d - 2 * l - r;
+            if ((unsigned)j >= (unsigned)T) {
+                e[r] = 0.f;
+                X[r] = 0.f;
+            }
+        }
+        const float u_o1 = __shfl_up_sync(0xffffffffu, X[1], 1);
+        const float u_e1 = __shfl_up_sync(0xffffffffu, X[0], 1);
+        const float u_o2 = __shfl_up_sync(0xffffffffu, X[1], 2);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i = 2 * l + r, j = d - i;
+            if ((unsigned)j < (unsigned)T) {
+                sm.Es[i][j] = e[r];
+                sm.XT[j][i] = X[r];
+                sm.Cs[i][j] = (int8_t)code[r];
+            }
+        }
+        tc::mbar_arrive(&sm.cbar[d % WS_RING]);
+        uo1_2 = uo1_1; uo1_1 = u_o1;
+        ue1_3 = ue1_2; ue1_2 = ue1_1; ue1_1 = u_e1;
+        uo2_3 = uo2_2; uo2_2 = uo2_1; uo2_1 = u_o2;
+        xe_1 = X[0];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            e3[r] = e2[r];
+            e2[r] = e1[r];
+            e1[r] = e[r];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) cpre[u] = npre[u];
+#pragma unroll
+        for (int u = 0; u < 5; ++u) {
+            ccol[0][u] = ncol[0][u];
+            ccol[1][u] = ncol[1][u];
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(WS_THREADS, 1)
+k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, float* __restrict__ Wt,
+          float* __restrict__ R, float* __restrict__ Ebuf, float* __restrict__ Elo, float* __restrict__ XTg,
+          float* __restrict__ XTlo, const float* __restrict__ UA, int64_t ldA, const float* __restrict__ UB,
+          int64_t ldB, const float* __restrict__ sp, int qmin, int qmax, int8_t* __restrict__ codes,
+          float* __restrict__ V, float* __restrict__ outE, DevStatus* status) {
+    constexpr int T = KG_T;
+    constexpr int VW = 4;
+    constexpr int NC = T / (4 * VW);   // chunks per lane and dot product
+    constexpr int A = WS_AHEAD;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    LeafWsSmem& sm = *reinterpret_cast<LeafWsSmem*>(smem_raw);
+
+    const int Imin = max(0, D - Nt + 1);
+    const int I = Imin + blockIdx.x;
+    const int J = D - I;
+    const int tid = threadIdx.x;
+    const bool helper = tid < WS_HELPERS;
+    const bool loader = tid < 256;     // threads that stage tiles and write back
+    const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
+
+    // ---- load: a^T (masked to k <= j-4) and the column constants, b row-major (masked) into
+    //      Es, R into XT, W~ into Ws
+    if (tid == 0) {
+        sm.abort_flag = 0;
+        for (int c = 0; c < 3; ++c)
+            for (int k = c; k < 3; ++k) sm.colc[c][k] = 0.f;   // a[j-k-1][j] with j-k-1 < 0
+    }
+    if (loader) {
+        leaf_load_tile<float, 1>(UA + c0 * ldA + c0, ldA, [&](int r, int c, float x) {
+            sm.aT[c][r] = (r <= c - A) ? x : 0.f;
+            if (r == c) {
+                sm.colc[c][4] = x;
+                sm.colc[c][3] = 1.f / x;
+            } else if (r == c - 1) {
+                sm.colc[c][0] = x;
+            } else if (r == c - 2) {
+                sm.colc[c][1] = x;
+            } else if (r == c - 3) {
+                sm.colc[c][2] = x;
+            }
+        });
+        leaf_load_tile<float, 1>(UB + r0 * ldB + r0, ldB, [&](int r, int c, float x) { sm.Es[r][c] = (c >= r) ? x : 0.f; });
+        leaf_load_tile<float, 1>(R + r0 * Np + c0, Np, [&](int r, int c, float x) { sm.XT[r][c] = x; });
+        leaf_load_tile<float, 1>(Wt + r0 * Np + c0, Np, [&](int r, int c, float x) { sm.Ws[r][c] = x; });
+        if (tid < T) {
+            const float s = sp[r0 + tid];
+            sm.s[tid] = s;
+            sm.invs[tid] = 1.f / s;
+        }
+    }
+    if (tid == 0) {
+        for (int k = 0; k < WS_RING; ++k) {
+            tc::mbar_init(&sm.cbar[k], 32);
+            tc::mbar_init(&sm.hbar[k], T);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // ---- per-row constants.  Helpers: U_B column of the row for k <= i-4 in registers.
+    //      Rounding warp: b_ii, b[i-1][i], b[i-2][i], b[i-3][i], s_i for its two rows.
+    const int ht = tid & 255, g = tid >> 8;
+    const int i = ht >> 2, q = ht & 3;
+    float breg[NC][VW];
+#pragma unroll
+    for (int t = 0; t < NC; ++t)
+#pragma unroll
+        for (int u = 0; u < VW; ++u) {
+            const int k = VW * q + 4 * VW * t + u;
+            breg[t][u] = (helper && k <= i - A) ? sm.Es[k][i] : 0.f;
+        }
+    float bii[2], b1[2], b2[2], b3[2], sr[2], isr[2], ib[2];
+    if (!helper) {
+        const int l = tid & 31;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int ir = 2 * l + r;
+            bii[r] = sm.Es[ir][ir];
+            b1[r] = (ir >= 1) ? sm.Es[ir - 1][ir] : 0.f;
+            b2[r] = (ir >= 2) ? sm.Es[ir - 2][ir] : 0.f;
+            b3[r] = (ir >= 3) ? sm.Es[ir - 3][ir] : 0.f;
+            sr[r] = sm.s[ir];
+            isr[r] = sm.invs[ir];
+            ib[r] = 1.f / bii[r];
+        }
+    }
+
+    // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i)
+    {
+        const int ty = (tid >> 4) & 15, tx = tid & 15;
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+        if (loader) {
+            const int kmax = ty * 4 + 3;
+#pragma unroll 4
+            for (int k = 0; k <= kmax; ++k) {
+                float bv[4], rv[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) bv[a] = sm.Es[k][ty * 4 + a];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) rv[c] = sm.XT[k][tx * 4 + c];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[a][c] += bv[a] * rv[c];
+            }
+        }
+        __syncthreads();
+        if (loader) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sm.Ws[ty * 4 + a][tx * 4 + c] -= acc[a][c];
+        }
+        // Es and XT start the sweep at zero (unvisited entries contribute nothing)
+        for (int idx = tid; idx < T * T; idx += WS_THREADS) {
+            sm.Es[idx / T][idx % T] = 0.f;
+            sm.XT[idx / T][idx % T] = 0.f;
+        }
+    }
+    __syncthreads();
+
+    // ---- sweep
+    const float fqmin = (float)qmin, fqmax = (float)qmax;
+    bool ok = true;
+    if (!helper) {
+        ok = ws_round_warp(sm, bii, b1, b2, b3, sr, isr, ib, fqmin, fqmax);
+    } else {
+        for (int d = g; d < 2 * T - 1; d += WS_GROUPS) {
+            if (d >= A) {
+                // step d needs everything published up to step d-4; lane 0 waits for the warp
+                const int dp = d - A;
+                bool w_ok = true;
+                if ((tid & 31) == 0)
+                    w_ok = tc::mbar_wait(&sm.cbar[dp % WS_RING], (uint32_t)((dp / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
+                                         &sm.abort_flag);
+                __syncwarp();   // orders lane 0's acquire before the other lanes' reads
+                w_ok = __shfl_sync(0xffffffffu, (int)w_ok, 0) != 0;
+                if (!w_ok) {
+                    ok = false;
+                    break;
+                }
+            }
+            const int j = d - i;
+            const bool active = (unsigned)j < (unsigned)T;
+            const int jr = active ? j : 0;
+            float4 xv[NC], av[NC], ev[NC];
+#pragma unroll
+            for (int t = 0; t < NC; ++t) {
+                const int k0 = VW * q + 4 * VW * t;
+                const bool pc = active && k0 <= i - A;
+                const bool pr = active && k0 <= j - A;
+                xv[t] = pc ? *reinterpret_cast<const float4*>(&sm.XT[jr][k0]) : float4{};
+                av[t] = pr ? *reinterpret_cast<const float4*>(&sm.aT[jr][k0]) : float4{};
+                ev[t] = pr ? *reinterpret_cast<const float4*>(&sm.Es[i][k0]) : float4{};
+            }
+            const float w = active ? sm.Ws[i][jr] : 0.f;
+            float c, r;
+            ws_dots(breg, xv, av, ev, c, r);
+            c += __shfl_xor_sync(0xffffffffu, c, 1);
+            r += __shfl_xor_sync(0xffffffffu, r, 1);
+            c += __shfl_xor_sync(0xffffffffu, c, 2);
+            r += __shfl_xor_sync(0xffffffffu, r, 2);
+            if (active && q == 0) {
+                sm.pre[d % WS_RING][i][0] = w - c;
+                sm.pre[d % WS_RING][i][1] = r;
+            }
+            if (q == 0) tc::mbar_arrive(&sm.hbar[d % WS_RING]);
+        }
+    }
+    if (!ok) {
+        sm.abort_flag = 1;   // wakes the other role out of its waits
+        set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
+    }
+    __syncthreads();
+    if (*reinterpret_cast<volatile int*>(&sm.abort_flag) != 0) return;
+
+    // ---- write back: codes, V = s_i code, E (16-byte stores where the layout allows)
+    constexpr int PER_ROW = T / VW;
+    if (loader) {
+        for (int f = tid; f < T * PER_ROW; f += 256) {
+            const int rr = f / PER_ROW, cc = (f % PER_ROW) * VW;
+            const int64_t gi = r0 + rr, gj = c0 + cc;
+            const float4 evv = *reinterpret_cast<const float4*>(&sm.Es[rr][cc]);
+            leaf_store_split(Ebuf, Elo, gi * Np + gj, evv);
+            if (gi < m) {
+                const float* es = reinterpret_cast<const float*>(&evv);
+#pragma unroll
+                for (int u = 0; u < VW; ++u) {
+                    if (gj + u < n) {
+                        codes[gi * n + gj + u] = sm.Cs[rr][cc + u];
+                        V[gi * n + gj + u] = (float)sm.Cs[rr][cc + u] * sm.s[rr];
+                        if (outE) outE[gi * n + gj + u] = es[u];
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    // ---- the complete X = R + local X: back into R (row-major) and into XTg (X transposed,
+    //      leading dimension Mp, split for the tensor-core update)
+    if (loader) leaf_load_tile<float, 1>(R + r0 * Np + c0, Np, [&](int rr, int cc, float x) { sm.XT[cc][rr] += x; });
+    __syncthreads();
+    if (loader && XTg) {
+        for (int f = tid; f < T * PER_ROW; f += 256) {
+            const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
+            leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
+        }
+    }
+    for (int idx = tid; idx < T * T; idx += WS_THREADS) {
+        const int cc = idx / T, rr = idx % T;
+        sm.Ws[rr][cc] = sm.XT[cc][rr];
+    }
+    __syncthreads();
+    if (loader) {
+        for (int f = tid; f < T * PER_ROW; f += 256) {
+            const int rr = f / PER_ROW, cc = (f % PER_ROW) * VW;
+            *reinterpret_cast<float4*>(R + (r0 + rr) * Np + c0 + cc) = *reinterpret_cast<const float4*>(&sm.Ws[rr][cc]);
+        }
+    }
+}
+
+}  // namespace kg

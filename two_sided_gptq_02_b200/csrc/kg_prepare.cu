@@ -177,8 +177,7 @@ k_syrk(double* __restrict__ M, int64_t kp, int kb) {
     Dmma64::zero(acc);
     Pipe::run(acc, sm, NB, M + (int64_t)ib * NB * kp + (int64_t)kb * NB, kp,
               M + (int64_t)jb * NB * kp + (int64_t)kb * NB, kp);
-    double* out = M + (int64_t)ib * NB * kp + (int64_t)jb * NB;
-    Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] -= v; });
+    Dmma64::add_to(acc, M + (int64_t)ib * NB * kp + (int64_t)jb * NB, kp, -1.0);
 }
 
 // X[ib,ib] = Dinv[ib] and zero the strictly upper block triangle of X

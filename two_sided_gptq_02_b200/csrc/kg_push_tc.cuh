@@ -233,32 +233,39 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
     if (!all_done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
     tc::fence_after_sync();
     if (all_done) {
+        // The whole 64-column accumulator row of this thread comes out of TMEM first; then all
+        // global loads of the read-modify-write are issued before any store, so the update costs
+        // one memory round trip rather than one per element.
         const int mrow = warp * 32 + lane;
         const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
         const bool valid = two || mrow < 64;
+        float v[PushTc::N];
 #pragma unroll
-        for (int cb = 0; cb < PushTc::N / 16; ++cb) {
-            float v[16];
-            tc::tmem_ld16(trow + cb * 16, v);
-            tc::tmem_wait_ld();
-            if (valid) {
-                if (chain == 1) {
-                    float* out = Wt + ((int64_t)I * T + mrow) * Np + (int64_t)J * T + cb * 16;
+        for (int cb = 0; cb < PushTc::N / 16; ++cb)
+            tc::tmem_ld16(trow + cb * 16, *reinterpret_cast<float(*)[16]>(&v[cb * 16]));
+        tc::tmem_wait_ld();
+        if (valid) {
+            if (chain == 1) {
+                float4* out = reinterpret_cast<float4*>(Wt + ((int64_t)I * T + mrow) * Np + (int64_t)J * T);
+                float4 o[PushTc::N / 4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float4 o = *reinterpret_cast<float4*>(out + 4 * q);
-                        o.x -= v[4 * q + 0];
-                        o.y -= v[4 * q + 1];
-                        o.z -= v[4 * q + 2];
-                        o.w -= v[4 * q + 3];
-                        *reinterpret_cast<float4*>(out + 4 * q) = o;
-                    }
-                } else {
-                    // D[m][n] = dR[I*64 + n][J*64 + m]
-                    float* out = R + ((int64_t)I * T + cb * 16) * Np + (int64_t)J * T + mrow;
+                for (int q = 0; q < PushTc::N / 4; ++q) o[q] = out[q];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) out[(int64_t)q * Np] += v[q];
+                for (int q = 0; q < PushTc::N / 4; ++q) {
+                    o[q].x -= v[4 * q + 0];
+                    o[q].y -= v[4 * q + 1];
+                    o[q].z -= v[4 * q + 2];
+                    o[q].w -= v[4 * q + 3];
+                    out[q] = o[q];
                 }
+            } else {
+                // D[m][n] = dR[I*64 + n][J*64 + m]: column m of the thread, one row per n
+                float* out = R + (int64_t)I * T * Np + (int64_t)J * T + mrow;
+                float o[PushTc::N];
+#pragma unroll
+                for (int q = 0; q < PushTc::N; ++q) o[q] = out[(int64_t)q * Np];
+#pragma unroll
+                for (int q = 0; q < PushTc::N; ++q) out[(int64_t)q * Np] = o[q] + v[q];
             }
         }
     }

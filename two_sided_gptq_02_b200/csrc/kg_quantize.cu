@@ -30,6 +30,7 @@
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
 #include "kg_leaf.cuh"
+#include "kg_leaf_ws.cuh"
 #include "kg_profile.cuh"
 #include "kg_push_tc.cuh"
 
@@ -174,45 +175,13 @@ k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
         if (k0 >= k1) return;
         PipeRow::run(acc, *reinterpret_cast<PipeRow::Smem*>(smem), (k1 - k0) * T,
                      E + (int64_t)I * T * Np + (int64_t)k0 * T, Np, UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA);
-        double* out = R + (int64_t)I * T * Np + (int64_t)J * T;
-        Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] += v; });
+        Dmma64::add_to(acc, R + (int64_t)I * T * Np + (int64_t)J * T, Np, 1.0);
     } else {
         const int k0 = max(0, D0 - J), k1 = min(Mt, mid - J);
         if (k0 >= k1) return;
         PipeCol::run(acc, *reinterpret_cast<PipeCol::Smem*>(smem), (k1 - k0) * T,
                      UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB, R + (int64_t)k0 * T * Np + (int64_t)J * T, Np);
-        double* out = Wt + (int64_t)I * T * Np + (int64_t)J * T;
-        Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * Np + c] -= v; });
-    }
-}
-
-__global__ void __launch_bounds__(Simt64f::kThreads)
-k_push_f32(int D0, int mid, int Mt, int Nt, int64_t Np,
-           float* __restrict__ Wt, float* __restrict__ R, const float* __restrict__ E,
-           const float* __restrict__ UA, int64_t ldA, const float* __restrict__ UB, int64_t ldB) {
-    __shared__ __align__(16) Simt64f::Smem sm;
-    const int D = mid + blockIdx.y;
-    const int I = max(0, D - Nt + 1) + blockIdx.x;
-    if (I > min(D, Mt - 1)) return;
-    const int J = D - I;
-    Simt64f::Acc acc;
-    Simt64f::zero(acc);
-    if (blockIdx.z == 0) {
-        const int k0 = max(0, D0 - I), k1 = min(Nt, mid - I);
-        if (k0 >= k1) return;
-        LdAf_RowMajor la{E + (int64_t)I * T * Np + (int64_t)k0 * T, Np};
-        LdBf_RowMajor lb{UA + (int64_t)k0 * T * ldA + (int64_t)J * T, ldA};
-        Simt64f::run(acc, sm, (k1 - k0) * T, la, lb);
-        float* out = R + (int64_t)I * T * Np + (int64_t)J * T;
-        Simt64f::for_each(acc, [&](int r, int c, float v) { out[(int64_t)r * Np + c] += v; });
-    } else {
-        const int k0 = max(0, D0 - J), k1 = min(Mt, mid - J);
-        if (k0 >= k1) return;
-        LdAf_Trans la{UB + (int64_t)k0 * T * ldB + (int64_t)I * T, ldB};
-        LdBf_RowMajor lb{R + (int64_t)k0 * T * Np + (int64_t)J * T, Np};
-        Simt64f::run(acc, sm, (k1 - k0) * T, la, lb);
-        float* out = Wt + (int64_t)I * T * Np + (int64_t)J * T;
-        Simt64f::for_each(acc, [&](int r, int c, float v) { out[(int64_t)r * Np + c] -= v; });
+        Dmma64::add_to(acc, Wt + (int64_t)I * T * Np + (int64_t)J * T, Np, -1.0);
     }
 }
 
@@ -240,11 +209,16 @@ static int launch_leaf(const QArgs<Real>& a, int D) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
     const int Imin = std::max(0, D - Nt + 1), Imax = std::min(D, Mt - 1);
     const int ntiles = Imax - Imin + 1;
-    const size_t smem = sizeof(LeafSmem<Real>);
     ProfScope ps(PK_LEAF, a.st);
-    k_leaf<Real><<<ntiles, 256, smem, a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT,
-                                              a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V,
-                                              a.outE);
+    if constexpr (sizeof(Real) == 4) {
+        k_leaf_ws<<<ntiles, WS_THREADS, sizeof(LeafWsSmem), a.st>>>(
+            D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB,
+            a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE, a.status);
+    } else {
+        k_leaf<Real><<<ntiles, 256, sizeof(LeafSmem<Real>), a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt,
+                                                                   a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB,
+                                                                   a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
+    }
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -386,16 +360,20 @@ static int configure_leaf() {
         // The solve alternates leaf and update launches.  All of them ask for the largest
         // shared-memory carveout, so the SMs never switch their L1 / shared split between two
         // launches of one solve.
-        KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(LeafSmem<Real>)));
-        KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<Real>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         cudaSharedmemCarveoutMaxShared));
         if (idx == 0) {
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_ws, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sizeof(LeafWsSmem)));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_ws, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              PushTc::SMEM_BYTES));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
         } else {
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)sizeof(LeafSmem<double>)));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<double>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_f64, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
         }
