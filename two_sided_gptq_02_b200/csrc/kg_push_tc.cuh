@@ -7,10 +7,12 @@
 //   row chain     R[I,J]  += sum_{J'} E[I,J'] U_A[J',J]            (J' over band 1 of row I)
 // Every fp32 operand x is kept as two tf32 planes hi + lo (x = hi + lo to ~22 bits); each product
 // is a_hi b_hi + a_hi b_lo + a_lo b_hi, accumulated in fp32 in tensor memory (TMEM).
-// Target tiles that share a K range are paired along M: two tiles of one column (column chain)
-// or, computing R^T = U_A^T E^T, two tiles of one row (row chain).  One CTA computes one 128 x 64
-// block with M=128, N=64, K=8 MMAs.  Both operands are read K-major (k contiguous) from split
-// copies the solve keeps for this purpose:
+// One CTA computes a 128 x 128 block with M=128, N=128, K=8 MMAs: two target tiles (M) against
+// two operand tiles (N) whose K ranges differ by one tile (adjacent columns of X in the column
+// chain; adjacent rows of E in the row chain, which computes R^T = U_A^T E^T).  The CTA runs over
+// the union of the two K ranges and loads the operand box of the one tile outside its range from
+// beyond the tensor, which the TMA fills with zeros; targets outside the band are not stored.
+// Both operands are read K-major (k contiguous) from split copies the solve keeps for this purpose:
 //   row chain     A(m,k) = U_A^T[J*64+m][k],   B(k,n) = E[I*64+n][k]      D[m][n] = dR[n][m]
 //   column chain  A(m,k) = U_B^T[I*64+m][k],   B(k,n) = X^T[J*64+n][k]    D[m][n] = dW[m][n]
 // Staging: a chunk is 32 K-elements, so each operand row is one 128-byte line; tensor-map loads
@@ -19,7 +21,7 @@
 //   * one producer thread (warp 0) issues the loads of a stage, completing on the stage's "full"
 //     mbarrier by transaction count;
 //   * one MMA thread (warp 1) waits for a full stage, issues its 12 MMAs and commits them to
-//     the stage's "empty" mbarrier, which the producer waits on before refilling it (4 stages);
+//     the stage's "empty" mbarrier, which the producer waits on before refilling it (3 stages);
 //   * all four warps meet only at the end, to drain the accumulator from TMEM.
 // Every wait is bounded in time and ends early once the solve has recorded an error; before the
 // CTA exits it waits (bounded, without early exit) for the loads it issued and the MMAs it
@@ -37,21 +39,30 @@
 
 namespace kg {
 
-struct PushTc {
-    static constexpr int M = 128, N = 64, BK = 32, STAGES = 4, THREADS = 128;
-    // one chunk = BK = 32 K-elements = one 128-byte line per operand row
+// NB operand tiles per CTA (N = 64 NB): NB = 2 pairs two operand tiles whose K ranges differ by
+// one tile and runs over their union; NB = 1 (small bands, where the extra tile would double the
+// work) takes one operand tile and its exact K range.
+template <int NB>
+struct PushCfg {
+    static constexpr int M = 128, N = 64 * NB, BK = 32, STAGES = NB == 2 ? 3 : 4, THREADS = 128;
+    // chunk = BK = 32 K-elements = one 128-byte line per operand row
     static constexpr int A_BYTES = M * BK * 4;                         // 16 KB per plane
-    static constexpr int B_BYTES = N * BK * 4;                         //  8 KB
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;      // 48 KB
+    static constexpr int B_BYTES = N * BK * 4;                         // 8 KB per plane per operand tile
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;      // 64 KB (NB = 2) or 48 KB
     static constexpr int BOX_BYTES = 64 * BK * 4;                      // one 64-row box of one plane
+    static constexpr int CHUNK_BYTES = (4 + 2 * NB) * BOX_BYTES;       // 2 target tiles x 2 planes + B
     // + barriers (full[S], empty[S], done), TMEM slot, counters; + pad to a 1024-byte base
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
-    static constexpr uint32_t TMEM_COLS = 64;
+    static constexpr uint32_t TMEM_COLS = N;
     // 128-byte swizzled K-major layout: rows of 128 bytes, 8-row groups 1024 bytes apart
     static constexpr uint32_t SBO = 1024;
+    // a row coordinate beyond every tensor map (m, n <= 2^20): loads there read zeros
+    static constexpr int OOB_ROW = 1 << 21;
     // about 0.1 s at 2 GHz: far beyond any legitimate wait for one stage of MMAs
     static constexpr long long MAX_WAIT_CYCLES = 200000000LL;
 };
+// the band (in K tiles) from which the update pairs operand tiles
+constexpr int PUSH_PAIR_MIN_K = 4;
 
 // Split operand planes of the tensor-core update (all fp32 values exactly representable as
 // tf32).  E* are Mp x Np (row-major), XT* Np x Mp, UAT* Np x Np, UBT* Mp x Mp.
@@ -60,7 +71,7 @@ struct SplitOperands {
 };
 
 // Tensor maps of the eight split planes (2-D, inner dimension = K, box 32 x 64, 128-byte
-// swizzle).  E* are Mp x Np, XT* Np x Mp, UAT* Np x Np, UBT* Mp x Mp (rows x inner).
+// swizzle, zero fill outside).  E* are Mp x Np, XT* Np x Mp, UAT* Np x Np, UBT* Mp x Mp (rows x inner).
 struct PushTmaMaps {
     CUtensorMap E_hi, E_lo, XT_hi, XT_lo, UAT_hi, UAT_lo, UBT_hi, UBT_lo;
 };
@@ -81,9 +92,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 }
 }  // namespace tc
 
-__global__ void __launch_bounds__(PushTc::THREADS, 1)
+template <int NB>
+__global__ void __launch_bounds__(PushCfg<NB>::THREADS, 1)
 k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restrict__ Wt, float* __restrict__ R,
             const __grid_constant__ PushTmaMaps maps, DevStatus* status) {
+    using PushTc = PushCfg<NB>;
     constexpr int T = KG_T;
     constexpr int S = PushTc::STAGES;
     extern __shared__ __align__(16) unsigned char smem_tc_raw[];
@@ -96,41 +109,30 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
     int* issued_s = reinterpret_cast<int*>(tslot + 1);     // chunks whose loads were issued
     int* consumed_s = issued_s + 1;                         // chunks whose MMAs were issued
 
-    const int chain = blockIdx.z;   // 0: row chain (into R), 1: column chain (into W~)
-    int I, J, k0, k1;
-    bool two;
-    if (chain == 1) {
-        J = blockIdx.x;
-        if (J >= Nt) return;
-        const int ilo = max(0, mid - J), ihi = min(Mt, D1 - J);
-        I = ilo + 2 * blockIdx.y;
-        if (I >= ihi) return;
-        two = (I + 1 < ihi);
-        k0 = max(0, D0 - J);
-        k1 = min(Mt, mid - J);
-    } else {
-        I = blockIdx.x;
-        if (I >= Mt) return;
-        const int jlo = max(0, mid - I), jhi = min(Nt, D1 - I);
-        J = jlo + 2 * blockIdx.y;
-        if (J >= jhi) return;
-        two = (J + 1 < jhi);
-        k0 = max(0, D0 - I);
-        k1 = min(Nt, mid - I);
-    }
+    // chain 1 (column chain, into W~): b = column J (B = X^T rows), t = row I (A = U_B^T rows),
+    //   K over rows I' of the source band.  chain 0 (row chain, into R, computed transposed):
+    //   b = row I (B = E rows), t = column J (A = U_A^T rows), K over columns J'.
+    // Tile (t, b) is a target when t + b lies in [mid, D1); operand tile b uses K tiles
+    // [D0 - b, mid - b).  The CTA takes b0, b0 + 1 and t0, t0 + 1 and runs over the union of the
+    // two K ranges; a B box outside its own range is loaded from beyond the tensor (zeros).
+    const int chain = blockIdx.z;
+    const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
+    const int b0 = NB * blockIdx.x;
+    if (b0 >= Bmax) return;
+    const int tlo = max(0, mid - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
+    const int t0 = tlo + 2 * blockIdx.y;
+    if (t0 >= thi) return;
+    const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
     if (k0 >= k1) return;
     // a solve that already failed (time-out, bad input) does no further tensor-core work
     if (*reinterpret_cast<const volatile int*>(&status->code) != 0) return;
     const int nchunks = (k1 - k0) * (T / PushTc::BK);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    const CUtensorMap* mAh = (chain == 1) ? &maps.UBT_hi : &maps.UAT_hi;
-    const CUtensorMap* mAl = (chain == 1) ? &maps.UBT_lo : &maps.UAT_lo;
-    const CUtensorMap* mBh = (chain == 1) ? &maps.XT_hi : &maps.E_hi;
-    const CUtensorMap* mBl = (chain == 1) ? &maps.XT_lo : &maps.E_lo;
-    const int rowA = (chain == 1) ? I * T : J * T;
-    const int rowB = (chain == 1) ? J * T : I * T;
-    const uint32_t chunk_bytes = (uint32_t)((two ? 4 : 2) + 2) * PushTc::BOX_BYTES;
+    const CUtensorMap* mAh = chain ? &maps.UBT_hi : &maps.UAT_hi;
+    const CUtensorMap* mAl = chain ? &maps.UBT_lo : &maps.UAT_lo;
+    const CUtensorMap* mBh = chain ? &maps.XT_hi : &maps.E_hi;
+    const CUtensorMap* mBl = chain ? &maps.XT_lo : &maps.E_lo;
 
     if (tid == 0) {
 #pragma unroll
@@ -142,18 +144,6 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
         *issued_s = 0;
         *consumed_s = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    // rows 64..127 of A stay zero in every stage when the pair is a single tile
-    if (!two) {
-        for (int s = 0; s < S; ++s) {
-            unsigned char* st = smem + s * PushTc::STAGE_BYTES;
-            for (int f = tid; f < PushTc::A_BYTES / 32; f += PushTc::THREADS) {
-                const int off = PushTc::A_BYTES / 2 + f * 16;
-                *reinterpret_cast<float4*>(st + off) = make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4*>(st + PushTc::A_BYTES + off) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-        tc::fence_proxy_async_smem();
     }
     if (warp == 0) {
         tc::tmem_alloc(tslot, PushTc::TMEM_COLS);
@@ -175,16 +165,22 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
                 break;
             }
             unsigned char* st = smem + s * PushTc::STAGE_BYTES;
-            const int kx = (k0 * T) + c * PushTc::BK;
-            tc::mbar_arrive_expect_tx(&full[s], chunk_bytes);
-            tc::tma_load_2d(st, mAh, kx, rowA, &full[s]);
-            tc::tma_load_2d(st + PushTc::A_BYTES, mAl, kx, rowA, &full[s]);
-            if (two) {
-                tc::tma_load_2d(st + PushTc::BOX_BYTES, mAh, kx, rowA + T, &full[s]);
-                tc::tma_load_2d(st + PushTc::A_BYTES + PushTc::BOX_BYTES, mAl, kx, rowA + T, &full[s]);
+            const int kt = k0 + c / (T / PushTc::BK);        // K tile of this chunk
+            const int kx = k0 * T + c * PushTc::BK;
+            tc::mbar_arrive_expect_tx(&full[s], PushTc::CHUNK_BYTES);
+            tc::tma_load_2d(st, mAh, kx, t0 * T, &full[s]);
+            tc::tma_load_2d(st + PushTc::BOX_BYTES, mAh, kx, (t0 + 1) * T, &full[s]);
+            tc::tma_load_2d(st + PushTc::A_BYTES, mAl, kx, t0 * T, &full[s]);
+            tc::tma_load_2d(st + PushTc::A_BYTES + PushTc::BOX_BYTES, mAl, kx, (t0 + 1) * T, &full[s]);
+            unsigned char* sb = st + 2 * PushTc::A_BYTES;
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                // B rows of operand tile b0 + u, or beyond the tensor when kt is outside its K range
+                const int b = b0 + u;
+                const int rb = (kt >= D0 - b && kt < mid - b) ? b * T : PushTc::OOB_ROW;
+                tc::tma_load_2d(sb + u * PushTc::BOX_BYTES, mBh, kx, rb, &full[s]);
+                tc::tma_load_2d(sb + PushTc::B_BYTES + u * PushTc::BOX_BYTES, mBl, kx, rb, &full[s]);
             }
-            tc::tma_load_2d(st + 2 * PushTc::A_BYTES, mBh, kx, rowB, &full[s]);
-            tc::tma_load_2d(st + 2 * PushTc::A_BYTES + PushTc::B_BYTES, mBl, kx, rowB, &full[s]);
             *reinterpret_cast<volatile int*>(issued_s) = c + 1;
         }
     } else if (warp == 1 && lane == 0) {
@@ -202,6 +198,7 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
             const uint32_t sb_hi = sa_hi + 2 * PushTc::A_BYTES, sb_lo = sb_hi + PushTc::B_BYTES;
 #pragma unroll
             for (int ks = 0; ks < PushTc::BK / 8; ++ks) {
+                // one MMA covers K = 8, i.e. 32 bytes of every row
                 const uint64_t ah = tc::smem_desc_sw128(sa_hi + 32 * ks, PushTc::SBO);
                 const uint64_t al = tc::smem_desc_sw128(sa_lo + 32 * ks, PushTc::SBO);
                 const uint64_t bh = tc::smem_desc_sw128(sb_hi + 32 * ks, PushTc::SBO);
@@ -233,25 +230,29 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
     if (!all_done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
     tc::fence_after_sync();
     if (all_done) {
-        // The whole 64-column accumulator row of this thread comes out of TMEM first; then all
-        // global loads of the read-modify-write are issued before any store, so the update costs
-        // one memory round trip rather than one per element.
+        // Thread mrow owns accumulator row mrow (target tile t = t0 + mrow / 64).  Each 64-column
+        // part (operand tile b = b0 + h) comes out of TMEM first; then all global loads of the
+        // read-modify-write are issued before any store (one memory round trip).
         const int mrow = warp * 32 + lane;
+        const int t = t0 + (mrow >> 6), r = mrow & 63;
         const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
-        const bool valid = two || mrow < 64;
-        float v[PushTc::N];
+#pragma unroll 1
+        for (int h = 0; h < NB; ++h) {
+            const int b = b0 + h;
+            float v[64];
 #pragma unroll
-        for (int cb = 0; cb < PushTc::N / 16; ++cb)
-            tc::tmem_ld16(trow + cb * 16, *reinterpret_cast<float(*)[16]>(&v[cb * 16]));
-        tc::tmem_wait_ld();
-        if (valid) {
+            for (int cb = 0; cb < 4; ++cb)
+                tc::tmem_ld16(trow + 64 * h + cb * 16, *reinterpret_cast<float(*)[16]>(&v[cb * 16]));
+            tc::tmem_wait_ld();
+            const bool valid = t < Tmax && b < Bmax && t + b >= mid && t + b < D1;
+            if (!valid) continue;
             if (chain == 1) {
-                float4* out = reinterpret_cast<float4*>(Wt + ((int64_t)I * T + mrow) * Np + (int64_t)J * T);
-                float4 o[PushTc::N / 4];
+                float4* out = reinterpret_cast<float4*>(Wt + ((int64_t)t * T + r) * Np + (int64_t)b * T);
+                float4 o[16];
 #pragma unroll
-                for (int q = 0; q < PushTc::N / 4; ++q) o[q] = out[q];
+                for (int q = 0; q < 16; ++q) o[q] = out[q];
 #pragma unroll
-                for (int q = 0; q < PushTc::N / 4; ++q) {
+                for (int q = 0; q < 16; ++q) {
                     o[q].x -= v[4 * q + 0];
                     o[q].y -= v[4 * q + 1];
                     o[q].z -= v[4 * q + 2];
@@ -259,13 +260,13 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
                     out[q] = o[q];
                 }
             } else {
-                // D[m][n] = dR[I*64 + n][J*64 + m]: column m of the thread, one row per n
-                float* out = R + (int64_t)I * T * Np + (int64_t)J * T + mrow;
-                float o[PushTc::N];
+                // D[m][n] = dR[b*64 + n][t*64 + r]: column r of target tile t, one row per n
+                float* out = R + (int64_t)b * T * Np + (int64_t)t * T + r;
+                float o[64];
 #pragma unroll
-                for (int q = 0; q < PushTc::N; ++q) o[q] = out[(int64_t)q * Np];
+                for (int q = 0; q < 64; ++q) o[q] = out[(int64_t)q * Np];
 #pragma unroll
-                for (int q = 0; q < PushTc::N; ++q) out[(int64_t)q * Np] = o[q] + v[q];
+                for (int q = 0; q < 64; ++q) out[(int64_t)q * Np] = o[q] + v[q];
             }
         }
     }
@@ -297,7 +298,7 @@ static bool push_tma_map(CUtensorMap* map, const float* base, int64_t inner, int
     if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (inner & 3) != 0) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)inner * sizeof(float)};
-    const cuuint32_t box[2] = {(cuuint32_t)PushTc::BK, 64u};
+    const cuuint32_t box[2] = {(cuuint32_t)PushCfg<1>::BK, 64u};
     const cuuint32_t estr[2] = {1u, 1u};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

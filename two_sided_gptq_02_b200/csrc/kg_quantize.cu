@@ -233,12 +233,18 @@ static int launch_push(const QArgs<double>& a, int D0, int mid, int D1) {
 }
 static int launch_push(const QArgs<float>& a, int D0, int mid, int D1) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    // one CTA per pair of target tiles sharing a K range: x = row (row chain) or column
-    // (column chain), y = pair index within it, z = chain
-    dim3 grid(std::max(Mt, Nt), (D1 - mid + 1) / 2, 2);
+    // one CTA per (operand tiles) x (target pair): x = operand tile or pair of them (columns of X
+    // in the column chain, rows of E in the row chain), y = target pair, z = chain
     ProfScope ps(PK_PUSH, a.st);
-    k_push_tc32<<<grid, PushTc::THREADS, PushTc::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt, a.R,
-                                                                      *a.maps, a.status);
+    if (mid - D0 >= PUSH_PAIR_MIN_K) {
+        dim3 grid((std::max(Mt, Nt) + 1) / 2, (D1 - mid + 2) / 2, 2);
+        k_push_tc32<2><<<grid, PushCfg<2>::THREADS, PushCfg<2>::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt,
+                                                                                 a.R, *a.maps, a.status);
+    } else {
+        dim3 grid(std::max(Mt, Nt), (D1 - mid + 1) / 2, 2);
+        k_push_tc32<1><<<grid, PushCfg<1>::THREADS, PushCfg<1>::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt,
+                                                                                 a.R, *a.maps, a.status);
+    }
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -365,9 +371,13 @@ static int configure_leaf() {
                                              (int)sizeof(LeafWsSmem)));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_ws, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
-            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             PushTc::SMEM_BYTES));
-            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32, cudaFuncAttributePreferredSharedMemoryCarveout,
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             PushCfg<1>::SMEM_BYTES));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             PushCfg<2>::SMEM_BYTES));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
         } else {
             KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf<double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
