@@ -47,6 +47,7 @@ def _args():
     ap.add_argument("--damp", type=float, default=0.01)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-block", action="store_true")
     return ap.parse_args()
 
 
@@ -139,6 +140,53 @@ def _leaf_flops(m, n):
     Mt, Nt = math.ceil(m / TILE), math.ceil(n / TILE)
     per_tile = 2 * (TILE * (TILE * (TILE - 1) // 2)) + TILE * (TILE * (TILE + 1) // 2)
     return 2.0 * per_tile * Mt * Nt
+
+
+def _block_seconds(kg, torch, damp, reps=3):
+    """The decoder-block workload: seven layers (q, k, v, o, gate, up, down), fp32, 3-bit,
+    quantized back to back -- once on one stream, once all seven in flight on one stream each.
+    Inputs are resident on the device; returns seconds per block (median of reps)."""
+    from synth_inputs.layers import layer_inputs, workload
+    specs = workload("block")
+    layers = []
+    for spec in specs:
+        W, A, B = layer_inputs(spec, device="cuda")
+        _, _, UA32, UB32 = kg.kron_gptq_prepare(A, B, damp)
+        W32 = W.float().contiguous()
+        s32 = kg.kron_gptq_row_scales(W32, spec.qmax)
+        del W, A, B
+        layers.append((spec, W32, UA32, UB32, s32, kg.Quantizer(spec.m, spec.n, torch.float32, "cuda")))
+    streams = [torch.cuda.Stream() for _ in layers]
+    main = torch.cuda.current_stream()
+
+    def one(concurrent):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(main)
+        for st, (spec, W32, UA32, UB32, s32, q) in zip(streams, layers):
+            st_use = st if concurrent else main
+            if concurrent:
+                st.wait_event(e0)
+            q.run(W32, UA32, UB32, s32, spec.qmin, spec.qmax, stream=st_use)
+        if concurrent:
+            for st in streams:
+                main.wait_stream(st)
+        e1.record(main)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    one(False)
+    one(True)
+    seq = statistics.median(one(False) for _ in range(reps))
+    con = statistics.median(one(True) for _ in range(reps))
+    for spec, *_, q in layers:
+        if q.status() != 0:
+            raise RuntimeError(f"block layer {spec.name}: status {q.status()}")
+    weights = sum(spec.m * spec.n for spec, *_ in layers)
+    return {"layers": [f"{spec.name} {spec.m}x{spec.n}" for spec, *_ in layers], "weights": weights,
+            "dtype": "f32", "bits": 3, "seconds_per_block_one_stream": seq,
+            "seconds_per_block_seven_streams": con, "weights_per_s_seven_streams": weights / con, "reps": reps,
+            "note": "inputs on the device; each layer its own seeded W, A, B (N=4096 rows); median of reps"}
 
 
 def _measure_dgemm_tflops(torch, dev):
@@ -374,6 +422,10 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": int(hW.numel() * es + hUA.numel() * es + hUB.numel() * es + hs.numel() * es),
                "d2h_bytes_per_step": int(hcodes.numel()), "ms_per_step": t_e2e / ke}
 
+    block = None
+    if rank == 0 and world == 1 and not args.no_block:
+        block = _block_seconds(kg, torch, args.damp)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(spec, W, A, B, args.damp)
@@ -390,6 +442,7 @@ def run_ours(args, rank, world, local_rank):
                                  f"{(bytes_compulsory + 3 * m * n * es) / 1e6:.0f} MB)"},
                 "roofline": rl, "roofline_other": rl_other, "solve_roofline": solve, "kernel_breakdown": breakdown,
                 "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
+                "block": block,
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
                           "source": peak_src}}
         print(json.dumps(line), flush=True)

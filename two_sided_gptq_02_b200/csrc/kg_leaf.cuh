@@ -47,6 +47,8 @@ struct LeafSmem {
     Real Es[KG_T][S];   // errors E[i][k]; during set-up b row-major
     Real XT[KG_T][S];   // local X transposed XT[j][k] = X[k][j]; during set-up R row-major
     Real Ws[KG_T][S];   // w', then Q
+    Real Rs[KG_T][KG_T + 1];   // R tile as loaded, then the transpose buffer for the final X
+                               // (stride 65: column and row walks are both conflict-free)
     Real s[KG_T], invs[KG_T], inva[KG_T], ajj[KG_T];
     int8_t Cs[KG_T][KG_T];
 };
@@ -75,33 +77,37 @@ __device__ __forceinline__ Real leaf_clamp(Real v, Real lo, Real hi) {
     return v < lo ? lo : (v > hi ? hi : v);
 }
 
-// Copy a 64x64 tile of a row-major matrix (leading dimension ld) into shared memory with a
-// per-element transform, issuing all 16-byte global loads of a pass before the stores.
+// Copy four 64x64 tiles of row-major matrices into shared memory with a per-element transform
+// store(tile, r, c, x), in PASSES memory round trips: each pass issues its share of the global
+// loads of all four tiles before any store.  Threads 0..255 take part.
 template <typename Real, int PASSES, class Store>
-__device__ __forceinline__ void leaf_load_tile(const Real* __restrict__ src, int64_t ld, Store store) {
+__device__ __forceinline__ void leaf_load_tiles4(const Real* const (&src)[4], const int64_t (&ld)[4], Store store) {
     constexpr int VW = LeafCfg<Real>::VW;
     constexpr int PER_ROW = KG_T / VW;                // vectors per tile row
-    constexpr int TOTAL = KG_T * PER_ROW;             // vectors per tile
-    constexpr int PER_THREAD = TOTAL / 256;           // 4 (fp32) or 8 (fp64)
+    constexpr int PER_THREAD = KG_T * PER_ROW / 256;  // per tile: 4 (fp32) or 8 (fp64)
     constexpr int PER_PASS = PER_THREAD / PASSES;
     using Vec = typename LeafCfg<Real>::V;
 #pragma unroll
     for (int p = 0; p < PASSES; ++p) {
-        Vec v[PER_PASS];
+        Vec v[4][PER_PASS];
 #pragma unroll
-        for (int e = 0; e < PER_PASS; ++e) {
-            const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
-            const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
-            v[e] = *reinterpret_cast<const Vec*>(src + (int64_t)r * ld + c);
-        }
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int e = 0; e < PER_PASS; ++e) {
-            const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
-            const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
-            const Real* x = reinterpret_cast<const Real*>(&v[e]);
+            for (int e = 0; e < PER_PASS; ++e) {
+                const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
+                const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+                v[t][e] = *reinterpret_cast<const Vec*>(src[t] + (int64_t)r * ld[t] + c);
+            }
 #pragma unroll
-            for (int u = 0; u < VW; ++u) store(r, c + u, x[u]);
-        }
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < PER_PASS; ++e) {
+                const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
+                const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+                const Real* x = reinterpret_cast<const Real*>(&v[t][e]);
+#pragma unroll
+                for (int u = 0; u < VW; ++u) store(t, r, c + u, x[u]);
+            }
     }
 }
 
@@ -127,13 +133,23 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
     const int tid = threadIdx.x;
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
-    // ---- load: a^T (masked), b row-major (masked) into Es, R into XT, W~ into Ws
-    leaf_load_tile<Real, PASSES>(UA + c0 * ldA + c0, ldA,
-                                 [&](int r, int c, Real x) { sm.aT[c][r] = (c >= r) ? x : Real(0); });
-    leaf_load_tile<Real, PASSES>(UB + r0 * ldB + r0, ldB,
-                                 [&](int r, int c, Real x) { sm.Es[r][c] = (c >= r) ? x : Real(0); });
-    leaf_load_tile<Real, PASSES>(R + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.XT[r][c] = x; });
-    leaf_load_tile<Real, PASSES>(Wt + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.Ws[r][c] = x; });
+    // ---- load: a^T (masked), b row-major (masked) into Es, R into XT (and Rs), W~ into Ws
+    {
+        const Real* const src[4] = {UA + c0 * ldA + c0, UB + r0 * ldB + r0, R + r0 * Np + c0, Wt + r0 * Np + c0};
+        const int64_t lds[4] = {ldA, ldB, Np, Np};
+        leaf_load_tiles4<Real, PASSES>(src, lds, [&](int t, int r, int c, Real x) {
+            if (t == 0) {
+                sm.aT[c][r] = (c >= r) ? x : Real(0);
+            } else if (t == 1) {
+                sm.Es[r][c] = (c >= r) ? x : Real(0);
+            } else if (t == 2) {
+                sm.XT[r][c] = x;
+                sm.Rs[r][c] = x;
+            } else {
+                sm.Ws[r][c] = x;
+            }
+        });
+    }
     if (tid < T) {
         const Real s = sp[r0 + tid];
         sm.s[tid] = s;
@@ -320,10 +336,13 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
             }
         }
     }
-    __syncthreads();
     // ---- the complete X = R + local X: back into R (row-major) and, when the tensor-core
-    //      update needs it, into XTg (X transposed, leading dimension Mp)
-    leaf_load_tile<Real, PASSES>(R + r0 * Np + c0, Np, [&](int r, int c, Real x) { sm.XT[c][r] += x; });
+    //      update needs it, into XTg (X transposed, leading dimension Mp), through the stride-65
+    //      buffer (independent of the write-back above: no barrier between them)
+    for (int idx = tid; idx < T * T; idx += 256) {
+        const int c = idx >> 6, r = idx & 63;
+        sm.XT[c][r] += sm.Rs[r][c];
+    }
     __syncthreads();
     constexpr int PER_ROW = T / VW;
     if (XTg) {
@@ -333,13 +352,13 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
         }
     }
     for (int idx = tid; idx < T * T; idx += 256) {
-        const int c = idx / T, r = idx % T;
-        sm.Ws[r][c] = sm.XT[c][r];
+        const int c = idx >> 6, r = idx & 63;
+        sm.Rs[r][c] = sm.XT[c][r];
     }
     __syncthreads();
-    for (int f = tid; f < T * PER_ROW; f += 256) {
-        const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
-        *reinterpret_cast<Vec*>(R + (r0 + r) * Np + c0 + c) = *reinterpret_cast<const Vec*>(&sm.Ws[r][c]);
+    for (int idx = tid; idx < T * T; idx += 256) {
+        const int r = idx >> 6, c = idx & 63;
+        R[(r0 + r) * Np + c0 + c] = sm.Rs[r][c];
     }
 }
 

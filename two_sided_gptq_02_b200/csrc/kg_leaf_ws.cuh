@@ -48,6 +48,8 @@ struct LeafWsSmem {
     float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
     float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
     float Ws[KG_T][S];             // w'
+    float Rs[KG_T][KG_T + 1];      // R tile as loaded, then the transpose buffer for the final X
+                                   // (stride 65: column and row walks are both conflict-free)
     float colc[KG_T][8];           // column j: a[j-1][j], a[j-2][j], a[j-3][j], 1/a[j][j], a[j][j]
     float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
     float s[KG_T], invs[KG_T];
@@ -185,7 +187,6 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     const int J = D - I;
     const int tid = threadIdx.x;
     const bool helper = tid < WS_HELPERS;
-    const bool loader = tid < 256;     // threads that stage tiles and write back
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
     // ---- load: a^T (masked to k <= j-4) and the column constants, b row-major (masked) into
@@ -195,23 +196,46 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
         for (int c = 0; c < 3; ++c)
             for (int k = c; k < 3; ++k) sm.colc[c][k] = 0.f;   // a[j-k-1][j] with j-k-1 < 0
     }
-    if (loader) {
-        leaf_load_tile<float, 1>(UA + c0 * ldA + c0, ldA, [&](int r, int c, float x) {
-            sm.aT[c][r] = (r <= c - A) ? x : 0.f;
-            if (r == c) {
-                sm.colc[c][4] = x;
-                sm.colc[c][3] = 1.f / x;
-            } else if (r == c - 1) {
-                sm.colc[c][0] = x;
-            } else if (r == c - 2) {
-                sm.colc[c][1] = x;
-            } else if (r == c - 3) {
-                sm.colc[c][2] = x;
+    if (helper) {
+        // the four tiles in one memory round trip: 512 threads x 8 float4, two of each tile
+        const float* src[4] = {UA + c0 * ldA + c0, UB + r0 * ldB + r0, R + r0 * Np + c0, Wt + r0 * Np + c0};
+        const int64_t lds[4] = {ldA, ldB, Np, Np};
+        float4 v[8];
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {
+            const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;   // e: vector index in the tile
+            v[f] = *reinterpret_cast<const float4*>(src[tile] + (int64_t)(e >> 4) * lds[tile] + (e & 15) * 4);
+        }
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {
+            const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;
+            const int r = e >> 4, c4 = (e & 15) * 4;
+            const float* x = reinterpret_cast<const float*>(&v[f]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = c4 + u;
+                if (tile == 0) {          // a: transposed, masked to k <= j-4; column constants
+                    sm.aT[c][r] = (r <= c - A) ? x[u] : 0.f;
+                    if (r == c) {
+                        sm.colc[c][4] = x[u];
+                        sm.colc[c][3] = 1.f / x[u];
+                    } else if (r == c - 1) {
+                        sm.colc[c][0] = x[u];
+                    } else if (r == c - 2) {
+                        sm.colc[c][1] = x[u];
+                    } else if (r == c - 3) {
+                        sm.colc[c][2] = x[u];
+                    }
+                } else if (tile == 1) {   // b row-major, masked to the upper triangle
+                    sm.Es[r][c] = (c >= r) ? x[u] : 0.f;
+                } else if (tile == 2) {   // R: for the fold (XT) and kept for the final X (Rs)
+                    sm.XT[r][c] = x[u];
+                    sm.Rs[r][c] = x[u];
+                } else {
+                    sm.Ws[r][c] = x[u];
+                }
             }
-        });
-        leaf_load_tile<float, 1>(UB + r0 * ldB + r0, ldB, [&](int r, int c, float x) { sm.Es[r][c] = (c >= r) ? x : 0.f; });
-        leaf_load_tile<float, 1>(R + r0 * Np + c0, Np, [&](int r, int c, float x) { sm.XT[r][c] = x; });
-        leaf_load_tile<float, 1>(Wt + r0 * Np + c0, Np, [&](int r, int c, float x) { sm.Ws[r][c] = x; });
+        }
         if (tid < T) {
             const float s = sp[r0 + tid];
             sm.s[tid] = s;
@@ -255,35 +279,31 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
         }
     }
 
-    // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i)
+    // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i);
+    //      512 threads, a 2 x 4 block each
     {
-        const int ty = (tid >> 4) & 15, tx = tid & 15;
-        float acc[4][4];
+        const int ty = tid >> 4, tx = tid & 15;   // rows 2 ty, 2 ty + 1; columns 4 tx .. 4 tx + 3
+        float acc[2][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 2; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-        if (loader) {
-            const int kmax = ty * 4 + 3;
+        if (helper) {
+            const int kmax = ty * 2 + 1;
 #pragma unroll 4
             for (int k = 0; k <= kmax; ++k) {
-                float bv[4], rv[4];
-#pragma unroll
-                for (int a = 0; a < 4; ++a) bv[a] = sm.Es[k][ty * 4 + a];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) rv[c] = sm.XT[k][tx * 4 + c];
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[a][c] += bv[a] * rv[c];
+                const float2 bv = *reinterpret_cast<const float2*>(&sm.Es[k][ty * 2]);
+                const float4 rv = *reinterpret_cast<const float4*>(&sm.XT[k][tx * 4]);
+                acc[0][0] += bv.x * rv.x; acc[0][1] += bv.x * rv.y; acc[0][2] += bv.x * rv.z; acc[0][3] += bv.x * rv.w;
+                acc[1][0] += bv.y * rv.x; acc[1][1] += bv.y * rv.y; acc[1][2] += bv.y * rv.z; acc[1][3] += bv.y * rv.w;
             }
         }
         __syncthreads();
-        if (loader) {
+        if (helper) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 2; ++a)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) sm.Ws[ty * 4 + a][tx * 4 + c] -= acc[a][c];
+                for (int c = 0; c < 4; ++c) sm.Ws[ty * 2 + a][tx * 4 + c] -= acc[a][c];
         }
         // Es and XT start the sweep at zero (unvisited entries contribute nothing)
         for (int idx = tid; idx < T * T; idx += WS_THREADS) {
@@ -350,8 +370,8 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 
     // ---- write back: codes, V = s_i code, E (16-byte stores where the layout allows)
     constexpr int PER_ROW = T / VW;
-    if (loader) {
-        for (int f = tid; f < T * PER_ROW; f += 256) {
+    if (helper) {
+        for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
             const int rr = f / PER_ROW, cc = (f % PER_ROW) * VW;
             const int64_t gi = r0 + rr, gj = c0 + cc;
             const float4 evv = *reinterpret_cast<const float4*>(&sm.Es[rr][cc]);
@@ -369,27 +389,30 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             }
         }
     }
-    __syncthreads();
-    // ---- the complete X = R + local X: back into R (row-major) and into XTg (X transposed,
-    //      leading dimension Mp, split for the tensor-core update)
-    if (loader) leaf_load_tile<float, 1>(R + r0 * Np + c0, Np, [&](int rr, int cc, float x) { sm.XT[cc][rr] += x; });
-    __syncthreads();
-    if (loader && XTg) {
-        for (int f = tid; f < T * PER_ROW; f += 256) {
-            const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
-            leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
-        }
-    }
+    // ---- the complete X = R + local X: into XTg (X transposed, leading dimension Mp, split for
+    //      the tensor-core update) and back into R (row-major), through the stride-65 buffer
+    //      (independent of the write-back above: no barrier between them)
     for (int idx = tid; idx < T * T; idx += WS_THREADS) {
-        const int cc = idx / T, rr = idx % T;
-        sm.Ws[rr][cc] = sm.XT[cc][rr];
+        const int cc = idx >> 6, rr = idx & 63;
+        sm.XT[cc][rr] += sm.Rs[rr][cc];
     }
     __syncthreads();
-    if (loader) {
-        for (int f = tid; f < T * PER_ROW; f += 256) {
-            const int rr = f / PER_ROW, cc = (f % PER_ROW) * VW;
-            *reinterpret_cast<float4*>(R + (r0 + rr) * Np + c0 + cc) = *reinterpret_cast<const float4*>(&sm.Ws[rr][cc]);
+    if (helper) {
+        if (XTg) {
+            for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
+                const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
+                leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
+            }
         }
+        for (int idx = tid; idx < T * T; idx += WS_HELPERS) {
+            const int cc = idx >> 6, rr = idx & 63;
+            sm.Rs[rr][cc] = sm.XT[cc][rr];
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < T * T; idx += WS_THREADS) {
+        const int rr = idx >> 6, cc = idx & 63;
+        R[(r0 + rr) * Np + c0 + cc] = sm.Rs[rr][cc];
     }
 }
 
