@@ -28,6 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+HERE = os.path.dirname(os.path.abspath(__file__))
 METRIC = "two-sided GPTQ weights/s & ms/layer (4096x4096, 3-bit) + % of roofline"
 TILE = 64
 # B200: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (max SM clock)
@@ -187,6 +188,29 @@ def _block_seconds(kg, torch, damp, reps=3):
             "dtype": "f32", "bits": 3, "seconds_per_block_one_stream": seq,
             "seconds_per_block_seven_streams": con, "weights_per_s_seven_streams": weights / con, "reps": reps,
             "note": "inputs on the device; each layer its own seeded W, A, B (N=4096 rows); median of reps"}
+
+
+def _traffic(kernel: str, units_per_launch: float):
+    """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/traffic.json):
+    bytes per unit of work (a tile for the leaves) x the units one launch processes on average.
+    None when there is no record or the kernel's source has changed since it was captured."""
+    import hashlib
+    path = os.path.join(HERE, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    src = os.path.join(HERE, rec["source"])
+    try:
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+    except OSError:
+        return None
+    return rec["dram_bytes_per_unit"] * units_per_launch
 
 
 def _measure_dgemm_tflops(torch, dev):
@@ -386,6 +410,9 @@ def run_ours(args, rank, world, local_rank):
                    "peak_source": "148 SMs x 64 FP64 lanes x 2 x 1.965 GHz"}
     for r_, ms_ in ((push_rl, pms), (leaf_rl, lms)):
         r_["ms_per_solve"] = ms_ / nprof
+    Mt_, Nt_ = math.ceil(m / TILE), math.ceil(n / TILE)
+    leaf_rl["traffic"] = _traffic(leaf_rl["kernel"], Mt_ * Nt_ / (ll / nprof))
+    leaf_rl["traffic_unit"] = "DRAM bytes per launch (ncu record x tiles per launch)"
     rl, rl_other = (push_rl, leaf_rl) if pms >= lms else (leaf_rl, push_rl)
     breakdown = {"push_ms_per_solve": pms / nprof, "leaf_ms_per_solve": lms / nprof, "init_ms_per_solve": ims / nprof,
                  "push_launches_per_solve": pl // nprof, "leaf_launches_per_solve": ll // nprof,

@@ -94,8 +94,8 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 template <int NB>
 __global__ void __launch_bounds__(PushCfg<NB>::THREADS, 1)
-k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restrict__ Wt, float* __restrict__ R,
-            const __grid_constant__ PushTmaMaps maps, DevStatus* status) {
+k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float* __restrict__ Wt,
+            float* __restrict__ R, const __grid_constant__ PushTmaMaps maps, DevStatus* status) {
     using PushTc = PushCfg<NB>;
     constexpr int T = KG_T;
     constexpr int S = PushTc::STAGES;
@@ -112,14 +112,14 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
     // chain 1 (column chain, into W~): b = column J (B = X^T rows), t = row I (A = U_B^T rows),
     //   K over rows I' of the source band.  chain 0 (row chain, into R, computed transposed):
     //   b = row I (B = E rows), t = column J (A = U_A^T rows), K over columns J'.
-    // Tile (t, b) is a target when t + b lies in [mid, D1); operand tile b uses K tiles
-    // [D0 - b, mid - b).  The CTA takes b0, b0 + 1 and t0, t0 + 1 and runs over the union of the
+    // Tile (t, b) is a target when t + b lies in [tgt0, D1) (tgt0 >= mid: the band may be updated
+    // in parts); operand tile b uses K tiles [D0 - b, mid - b).  The CTA takes b0, b0 + 1 and t0, t0 + 1 and runs over the union of the
     // two K ranges; a B box outside its own range is loaded from beyond the tensor (zeros).
     const int chain = blockIdx.z;
     const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
     const int b0 = NB * blockIdx.x;
     if (b0 >= Bmax) return;
-    const int tlo = max(0, mid - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
+    const int tlo = max(0, tgt0 - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
     const int t0 = tlo + 2 * blockIdx.y;
     if (t0 >= thi) return;
     const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
@@ -244,7 +244,7 @@ k_push_tc32(int D0, int mid, int D1, int Mt, int Nt, int64_t Np, float* __restri
             for (int cb = 0; cb < 4; ++cb)
                 tc::tmem_ld16(trow + 64 * h + cb * 16, *reinterpret_cast<float(*)[16]>(&v[cb * 16]));
             tc::tmem_wait_ld();
-            const bool valid = t < Tmax && b < Bmax && t + b >= mid && t + b < D1;
+            const bool valid = t < Tmax && b < Bmax && t + b >= tgt0 && t + b < D1;
             if (!valid) continue;
             if (chain == 1) {
                 float4* out = reinterpret_cast<float4*>(Wt + ((int64_t)t * T + r) * Np + (int64_t)b * T);

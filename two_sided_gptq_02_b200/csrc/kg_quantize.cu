@@ -26,6 +26,7 @@
 //             Both are dense GEMMs over contiguous K ranges.
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
@@ -153,10 +154,11 @@ __global__ void k_check_diag2(const Real* __restrict__ UA, int64_t n, const Real
 }
 
 // ------------------------------------------------------------------------------ push
-// Grid: x = position along a target diagonal, y = target diagonal offset from mid,
-// z = chain (0: row chain into R, 1: column chain into W~).
+// Sources: diagonals [D0, mid); targets: diagonals [tgt0, D1) with tgt0 >= mid (a band may be
+// updated in parts).  Grid: x = position along a target diagonal, y = target diagonal offset from
+// tgt0, z = chain (0: row chain into R, 1: column chain into W~).
 __global__ void __launch_bounds__(Dmma64::kThreads)
-k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
+k_push_f64(int D0, int mid, int tgt0, int Mt, int Nt, int64_t Np,
            double* __restrict__ Wt, double* __restrict__ R, const double* __restrict__ E,
            const double* __restrict__ UA, int64_t ldA, const double* __restrict__ UB, int64_t ldB) {
     using PipeRow = DmmaPipe<false, false>;   // A = rows of E,  B = rows of U_A
@@ -164,7 +166,7 @@ k_push_f64(int D0, int mid, int Mt, int Nt, int64_t Np,
     constexpr size_t kSmem = sizeof(PipeRow::Smem) > sizeof(PipeCol::Smem) ? sizeof(PipeRow::Smem)
                                                                             : sizeof(PipeCol::Smem);
     __shared__ __align__(16) unsigned char smem[kSmem];
-    const int D = mid + blockIdx.y;
+    const int D = tgt0 + blockIdx.y;
     const int I = max(0, D - Nt + 1) + blockIdx.x;
     if (I > min(D, Mt - 1)) return;
     const int J = D - I;
@@ -205,59 +207,151 @@ struct QArgs {
 };
 
 template <typename Real>
-static int launch_leaf(const QArgs<Real>& a, int D) {
+static int launch_leaf(const QArgs<Real>& a, int D, cudaStream_t st) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
     const int Imin = std::max(0, D - Nt + 1), Imax = std::min(D, Mt - 1);
     const int ntiles = Imax - Imin + 1;
-    ProfScope ps(PK_LEAF, a.st);
+    ProfScope ps(PK_LEAF, st);
     if constexpr (sizeof(Real) == 4) {
-        k_leaf_ws<<<ntiles, WS_THREADS, sizeof(LeafWsSmem), a.st>>>(
+        k_leaf_ws<<<ntiles, WS_THREADS, sizeof(LeafWsSmem), st>>>(
             D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB,
             a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE, a.status);
     } else {
-        k_leaf<Real><<<ntiles, 256, sizeof(LeafSmem<Real>), a.st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt,
-                                                                   a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB,
-                                                                   a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
+        k_leaf<Real><<<ntiles, 256, sizeof(LeafSmem<Real>), st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt,
+                                                                 a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB,
+                                                                 a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
     }
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
 
-static int launch_push(const QArgs<double>& a, int D0, int mid, int D1) {
+// Update of the targets on diagonals [tgt0, D1) from the sources on diagonals [D0, mid).
+static int launch_push(const QArgs<double>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    dim3 grid(std::min(Mt, Nt), D1 - mid, 2);
-    ProfScope ps(PK_PUSH, a.st);
-    k_push_f64<<<grid, Dmma64::kThreads, 0, a.st>>>(D0, mid, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB, a.ldB);
+    dim3 grid(std::min(Mt, Nt), D1 - tgt0, 2);
+    ProfScope ps(PK_PUSH, st);
+    k_push_f64<<<grid, Dmma64::kThreads, 0, st>>>(D0, mid, tgt0, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB,
+                                                  a.ldB);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
-static int launch_push(const QArgs<float>& a, int D0, int mid, int D1) {
+static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
     // one CTA per (operand tiles) x (target pair): x = operand tile or pair of them (columns of X
     // in the column chain, rows of E in the row chain), y = target pair, z = chain
-    ProfScope ps(PK_PUSH, a.st);
+    ProfScope ps(PK_PUSH, st);
     if (mid - D0 >= PUSH_PAIR_MIN_K) {
-        dim3 grid((std::max(Mt, Nt) + 1) / 2, (D1 - mid + 2) / 2, 2);
-        k_push_tc32<2><<<grid, PushCfg<2>::THREADS, PushCfg<2>::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt,
-                                                                                 a.R, *a.maps, a.status);
+        dim3 grid((std::max(Mt, Nt) + 1) / 2, (D1 - tgt0 + 2) / 2, 2);
+        k_push_tc32<2><<<grid, PushCfg<2>::THREADS, PushCfg<2>::SMEM_BYTES, st>>>(D0, mid, tgt0, D1, Mt, Nt, a.L.Np,
+                                                                               a.Wt, a.R, *a.maps, a.status);
     } else {
-        dim3 grid(std::max(Mt, Nt), (D1 - mid + 1) / 2, 2);
-        k_push_tc32<1><<<grid, PushCfg<1>::THREADS, PushCfg<1>::SMEM_BYTES, a.st>>>(D0, mid, D1, Mt, Nt, a.L.Np, a.Wt,
-                                                                                 a.R, *a.maps, a.status);
+        dim3 grid(std::max(Mt, Nt), (D1 - tgt0 + 1) / 2, 2);
+        k_push_tc32<1><<<grid, PushCfg<1>::THREADS, PushCfg<1>::SMEM_BYTES, st>>>(D0, mid, tgt0, D1, Mt, Nt, a.L.Np,
+                                                                               a.Wt, a.R, *a.maps, a.status);
     }
     KG_LAUNCH_CHECK();
+    return KG_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Two-stream schedule.  Every update push(D0 | mid | D1) is split: its targets on diagonal mid --
+// all the next leaf needs -- go on the caller's stream (the critical path); its targets on
+// diagonals (mid, D1) go on a second stream, where they overlap the leaves that follow (a leaf
+// occupies at most min(Mt, Nt) SMs).  (Splitting that rest further, into pieces of 1, 2, 4, ...
+// diagonals, measured slower: the pieces run less efficiently and contend with the leaves.)  Hazards are tracked per diagonal: a bulk update targeting
+// diagonal d records an event, and the first kernel on the critical stream that touches d waits
+// for the latest such event (the bulk stream runs in order, so that covers all earlier ones).
+// Bulk updates read only sources solved before the fork event that precedes them, and they never
+// target a diagonal the critical stream has already reached.  The caller's stream waits for the
+// bulk stream at the end.
+// ---------------------------------------------------------------------------------------
+struct Sched {
+    cudaStream_t crit, bulk;
+    cudaEvent_t fork;           // re-recorded before every bulk update (waits snapshot it)
+    cudaEvent_t* done;          // ring of events recorded after bulk updates, slot = seq % ndone
+    int ndone;
+    std::vector<int> pending;   // per diagonal: sequence number of the latest bulk update targeting it
+    int seq = -1;               // sequence number of the latest bulk update
+    int waited = -1;            // latest bulk update the critical stream has waited for
+};
+
+// The critical stream is about to touch diagonals [d0, d1): wait for the latest bulk update that
+// targets one of them.  A ring slot may since have been re-recorded by a later bulk update; the
+// wait then covers that later one too, which is conservative and cannot deadlock (bulk updates
+// wait only on fork events recorded earlier on the critical stream).
+static int sched_wait(Sched& s, int d0, int d1) {
+    int need = -1;
+    for (int d = d0; d < d1; ++d) need = std::max(need, s.pending[d]);
+    if (need > s.waited) {
+        KG_CUDA_TRY(cudaStreamWaitEvent(s.crit, s.done[need % s.ndone], 0));
+        s.waited = need;
+    }
     return KG_OK;
 }
 
 template <typename Real>
-static int solve_range(const QArgs<Real>& a, int D0, int D1) {
-    if (D1 - D0 == 1) return launch_leaf(a, D0);
+static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
+    int rc;
+    if (D1 - D0 == 1) {
+        if ((rc = sched_wait(s, D0, D0 + 1))) return rc;
+        return launch_leaf(a, D0, s.crit);
+    }
     const int mid = (D0 + D1) / 2;
-    int rc = solve_range(a, D0, mid);
+    if ((rc = solve_range(a, s, D0, mid))) return rc;
+    if ((rc = sched_wait(s, mid, mid + 1))) return rc;
+    if ((rc = launch_push(a, D0, mid, mid, mid + 1, s.crit))) return rc;
+    if (D1 > mid + 1) {
+        KG_CUDA_TRY(cudaEventRecord(s.fork, s.crit));
+        KG_CUDA_TRY(cudaStreamWaitEvent(s.bulk, s.fork, 0));
+        if ((rc = launch_push(a, D0, mid, mid + 1, D1, s.bulk))) return rc;
+        ++s.seq;
+        KG_CUDA_TRY(cudaEventRecord(s.done[s.seq % s.ndone], s.bulk));
+        for (int d = mid + 1; d < D1; ++d) s.pending[d] = s.seq;
+    }
+    return solve_range(a, s, mid, D1);
+}
+
+// Per host thread and device: the bulk stream and its events, created on first use and kept for
+// the life of the process.
+struct SchedPool {
+    int dev = -1;
+    cudaStream_t bulk = nullptr;
+    cudaEvent_t fork = nullptr;
+    std::vector<cudaEvent_t> done;
+};
+static constexpr int kSchedDone = 64;
+
+static int sched_pool(SchedPool*& out) {
+    static thread_local std::vector<SchedPool> pools;
+    int dev = 0;
+    KG_CUDA_TRY(cudaGetDevice(&dev));
+    for (auto& p : pools)
+        if (p.dev == dev) {
+            out = &p;
+            return KG_OK;
+        }
+    SchedPool p;
+    p.dev = dev;
+    KG_CUDA_TRY(cudaStreamCreateWithFlags(&p.bulk, cudaStreamNonBlocking));
+    KG_CUDA_TRY(cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming));
+    p.done.resize(kSchedDone);
+    for (auto& e : p.done) KG_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    pools.push_back(std::move(p));
+    out = &pools.back();
+    return KG_OK;
+}
+
+template <typename Real>
+static int solve_all(const QArgs<Real>& a, int ndiag) {
+    SchedPool* pool = nullptr;
+    int rc = sched_pool(pool);
     if (rc) return rc;
-    rc = launch_push(a, D0, mid, D1);
-    if (rc) return rc;
-    return solve_range(a, mid, D1);
+    Sched s{a.st, pool->bulk, pool->fork, pool->done.data(), (int)pool->done.size(), std::vector<int>(ndiag + 1, -1)};
+    rc = solve_range(a, s, 0, ndiag);
+    // join: the caller's stream waits for the last bulk update (also on the error path, so the
+    // bulk stream never runs past the caller's view of the solve)
+    if (s.seq > s.waited) KG_CUDA_TRY(cudaStreamWaitEvent(s.crit, s.done[s.seq % s.ndone], 0));
+    return rc;
 }
 
 template <typename Real>
@@ -348,7 +442,7 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         }
         KG_LAUNCH_CHECK();
     }
-    return solve_range(a, 0, (int)(L.Mt + L.Nt - 1));
+    return solve_all(a, (int)(L.Mt + L.Nt - 1));
 }
 
 // Kernel attributes are per device: configure each device once (guarded by a mutex).
