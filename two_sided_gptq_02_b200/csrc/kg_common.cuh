@@ -48,4 +48,12 @@ struct Vec2<float> { using type = float2; };
 template <>
 struct Vec2<double> { using type = double2; };
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the previous kernel of its stream is still running: it must call grid_dep_wait()
+// before touching anything that kernel writes (the wait returns once it has completed and its
+// memory is visible; without the launch attribute it returns at once).  grid_dep_launch() lets the
+// next kernel of the stream start launching early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace kg

@@ -134,6 +134,9 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
     // ---- load: a^T (masked), b row-major (masked) into Es, R into XT (and Rs), W~ into Ws
+    //      (after the previous kernel of the stream has finished: programmatic launch)
+    grid_dep_launch();
+    grid_dep_wait();
     {
         const Real* const src[4] = {UA + c0 * ldA + c0, UB + r0 * ldB + r0, R + r0 * Np + c0, Wt + r0 * Np + c0};
         const int64_t lds[4] = {ldA, ldB, Np, Np};

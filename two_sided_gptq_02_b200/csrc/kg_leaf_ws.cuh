@@ -187,6 +187,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     const int J = D - I;
     const int tid = threadIdx.x;
     const bool helper = tid < WS_HELPERS;
+    grid_dep_launch();
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
     // ---- load: a^T (masked to k <= j-4) and the column constants, b row-major (masked) into
@@ -203,6 +204,9 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
         float4 v[8];
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
+            // the factor tiles (f < 4) do not depend on earlier kernels of the solve: they load while
+            // the previous kernel finishes; R and W~ (f >= 4) only after it has
+            if (f == 4) grid_dep_wait();
             const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;   // e: vector index in the tile
             v[f] = *reinterpret_cast<const float4*>(src[tile] + (int64_t)(e >> 4) * lds[tile] + (e & 15) * 4);
         }

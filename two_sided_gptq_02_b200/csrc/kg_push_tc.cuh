@@ -124,8 +124,9 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     if (t0 >= thi) return;
     const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
     if (k0 >= k1) return;
-    // a solve that already failed (time-out, bad input) does no further tensor-core work
-    if (*reinterpret_cast<const volatile int*>(&status->code) != 0) return;
+    grid_dep_launch();
+    // set-up below overlaps the end of the previous kernel of the stream (programmatic launch);
+    // everything that kernel writes -- the status word included -- is read after grid_dep_wait()
     const int nchunks = (k1 - k0) * (T / PushTc::BK);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -153,11 +154,15 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tslot;
+    grid_dep_wait();
+    // a solve that already failed (time-out, bad input) does no further tensor-core work
+    const bool failed = *reinterpret_cast<const volatile int*>(&status->code) != 0;
+    const int nch = failed ? 0 : nchunks;
     bool ok = true;
 
     if (warp == 0 && lane == 0) {
         // ---- producer
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < nch; ++c) {
             const int s = c % S;
             if (c >= S && !tc::mbar_wait(&empty[s], (uint32_t)(((c / S) - 1) & 1), PushTc::MAX_WAIT_CYCLES,
                                          &status->code)) {
@@ -186,7 +191,7 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer
         const uint32_t idesc = tc::idesc_tf32(PushTc::M, PushTc::N, false, false);
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < nch; ++c) {
             const int s = c % S;
             if (!tc::mbar_wait(&full[s], (uint32_t)((c / S) & 1), PushTc::MAX_WAIT_CYCLES, &status->code)) {
                 ok = false;
@@ -226,10 +231,10 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
             drained &= tc::mbar_wait(&full[c % S], (uint32_t)((c / S) & 1), PushTc::MAX_WAIT_CYCLES, &never);
     }
     const bool all_done = __syncthreads_and(drained) &&
-                          *reinterpret_cast<volatile int*>(consumed_s) == nchunks;
+                          *reinterpret_cast<volatile int*>(consumed_s) == nch;
     if (!all_done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
     tc::fence_after_sync();
-    if (all_done) {
+    if (all_done && !failed) {
         // Thread mrow owns accumulator row mrow (target tile t = t0 + mrow / 64).  Each 64-column
         // part (operand tile b = b0 + h) comes out of TMEM first; then all global loads of the
         // read-modify-write are issued before any store (one memory round trip).

@@ -26,6 +26,7 @@
 //             Both are dense GEMMs over contiguous K ranges.
 #include <algorithm>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "kg_common.cuh"
@@ -170,6 +171,8 @@ k_push_f64(int D0, int mid, int tgt0, int Mt, int Nt, int64_t Np,
     const int I = max(0, D - Nt + 1) + blockIdx.x;
     if (I > min(D, Mt - 1)) return;
     const int J = D - I;
+    grid_dep_launch();
+    grid_dep_wait();   // programmatic launch: the previous kernel's writes are visible from here
     Dmma64::Acc acc;
     Dmma64::zero(acc);
     if (blockIdx.z == 0) {
@@ -206,6 +209,24 @@ struct QArgs {
     const PushTmaMaps* maps;
 };
 
+// Launch with programmatic stream serialization when pdl is set: the kernel may start while the
+// previous kernel of the stream finishes, and waits for it inside (grid_dep_wait).
+template <typename... KArgs, typename... Args>
+static int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                    Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? KG_OK : KG_ERR_CUDA;
+}
+
 template <typename Real>
 static int launch_leaf(const QArgs<Real>& a, int D, cudaStream_t st) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
@@ -213,44 +234,37 @@ static int launch_leaf(const QArgs<Real>& a, int D, cudaStream_t st) {
     const int ntiles = Imax - Imin + 1;
     ProfScope ps(PK_LEAF, st);
     if constexpr (sizeof(Real) == 4) {
-        k_leaf_ws<<<ntiles, WS_THREADS, sizeof(LeafWsSmem), st>>>(
-            D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB,
-            a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE, a.status);
+        return launch_k(k_leaf_ws, dim3(ntiles), dim3(WS_THREADS), sizeof(LeafWsSmem), st, true, D, Mt, Nt, a.L.m,
+                        a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp,
+                        a.qmin, a.qmax, a.codes, a.V, a.outE, a.status);
     } else {
-        k_leaf<Real><<<ntiles, 256, sizeof(LeafSmem<Real>), st>>>(D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt,
-                                                                 a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB,
-                                                                 a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.V, a.outE);
+        return launch_k(k_leaf<Real>, dim3(ntiles), dim3(256), sizeof(LeafSmem<Real>), st, true, D, Mt, Nt, a.L.m,
+                        a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp,
+                        a.qmin, a.qmax, a.codes, a.V, a.outE);
     }
-    KG_LAUNCH_CHECK();
-    return KG_OK;
 }
 
 // Update of the targets on diagonals [tgt0, D1) from the sources on diagonals [D0, mid).
-static int launch_push(const QArgs<double>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st) {
+static int launch_push(const QArgs<double>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st, bool pdl) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    dim3 grid(std::min(Mt, Nt), D1 - tgt0, 2);
     ProfScope ps(PK_PUSH, st);
-    k_push_f64<<<grid, Dmma64::kThreads, 0, st>>>(D0, mid, tgt0, Mt, Nt, a.L.Np, a.Wt, a.R, a.E, a.UA, a.ldA, a.UB,
-                                                  a.ldB);
-    KG_LAUNCH_CHECK();
-    return KG_OK;
+    return launch_k(k_push_f64, dim3(std::min(Mt, Nt), D1 - tgt0, 2), dim3(Dmma64::kThreads), 0, st, pdl, D0, mid,
+                    tgt0, Mt, Nt, a.L.Np, a.Wt, a.R, (const double*)a.E, a.UA, a.ldA, a.UB, a.ldB);
 }
-static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st) {
+static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st, bool pdl) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
     // one CTA per (operand tiles) x (target pair): x = operand tile or pair of them (columns of X
     // in the column chain, rows of E in the row chain), y = target pair, z = chain
     ProfScope ps(PK_PUSH, st);
-    if (mid - D0 >= PUSH_PAIR_MIN_K) {
-        dim3 grid((std::max(Mt, Nt) + 1) / 2, (D1 - tgt0 + 2) / 2, 2);
-        k_push_tc32<2><<<grid, PushCfg<2>::THREADS, PushCfg<2>::SMEM_BYTES, st>>>(D0, mid, tgt0, D1, Mt, Nt, a.L.Np,
-                                                                               a.Wt, a.R, *a.maps, a.status);
-    } else {
-        dim3 grid(std::max(Mt, Nt), (D1 - tgt0 + 1) / 2, 2);
-        k_push_tc32<1><<<grid, PushCfg<1>::THREADS, PushCfg<1>::SMEM_BYTES, st>>>(D0, mid, tgt0, D1, Mt, Nt, a.L.Np,
-                                                                               a.Wt, a.R, *a.maps, a.status);
-    }
-    KG_LAUNCH_CHECK();
-    return KG_OK;
+    // pairs of operand tiles for wide bands with several target diagonals; one target diagonal
+    // (the critical part) keeps one operand tile per CTA for twice the CTAs
+    if (mid - D0 >= PUSH_PAIR_MIN_K && D1 - tgt0 > 1)
+        return launch_k(k_push_tc32<2>, dim3((std::max(Mt, Nt) + 1) / 2, (D1 - tgt0 + 2) / 2, 2),
+                        dim3(PushCfg<2>::THREADS), PushCfg<2>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt,
+                        a.L.Np, a.Wt, a.R, *a.maps, a.status);
+    return launch_k(k_push_tc32<1>, dim3(std::max(Mt, Nt), (D1 - tgt0 + 1) / 2, 2), dim3(PushCfg<1>::THREADS),
+                    PushCfg<1>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps,
+                    a.status);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -299,11 +313,11 @@ static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
     const int mid = (D0 + D1) / 2;
     if ((rc = solve_range(a, s, D0, mid))) return rc;
     if ((rc = sched_wait(s, mid, mid + 1))) return rc;
-    if ((rc = launch_push(a, D0, mid, mid, mid + 1, s.crit))) return rc;
+    if ((rc = launch_push(a, D0, mid, mid, mid + 1, s.crit, true))) return rc;
     if (D1 > mid + 1) {
         KG_CUDA_TRY(cudaEventRecord(s.fork, s.crit));
         KG_CUDA_TRY(cudaStreamWaitEvent(s.bulk, s.fork, 0));
-        if ((rc = launch_push(a, D0, mid, mid + 1, D1, s.bulk))) return rc;
+        if ((rc = launch_push(a, D0, mid, mid + 1, D1, s.bulk, false))) return rc;
         ++s.seq;
         KG_CUDA_TRY(cudaEventRecord(s.done[s.seq % s.ndone], s.bulk));
         for (int d = mid + 1; d < D1; ++d) s.pending[d] = s.seq;
