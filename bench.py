@@ -421,33 +421,69 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end: host buffers through the same public call
     e2e = None
     if not args.no_e2e:
+        # A user pipeline with host buffers through the public call: every step copies its inputs
+        # (W, U_A, U_B, scales) host -> device from pinned memory, solves, and copies its codes
+        # device -> host; step k+1's inputs travel while step k solves (two device input sets, one
+        # stream per copy direction), and step k's codes travel while step k+1 solves.
         hW = Wd.cpu().pin_memory()
         hUA, hUB, hs = UAd.cpu().pin_memory(), UBd.cpu().pin_memory(), sd.cpu().pin_memory()
-        dW, dUA, dUB, ds = torch.empty_like(Wd), torch.empty_like(UAd), torch.empty_like(UBd), torch.empty_like(sd)
-        hcodes = torch.empty(m, n, dtype=torch.int8).pin_memory()
-        ke = max(1, min(args.steps, 5))
+        nb = 2
+        bufs = [(torch.empty_like(Wd), torch.empty_like(UAd), torch.empty_like(UBd), torch.empty_like(sd))
+                for _ in range(nb)]
+        qs = [kg.Quantizer(m, n, dt, dev) for _ in range(nb)]
+        hcodes = [torch.empty(m, n, dtype=torch.int8).pin_memory() for _ in range(nb)]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(nb)]      # inputs of set b on the device
+        ev_used = [torch.cuda.Event() for _ in range(nb)]    # solve on set b finished (inputs free)
+        ev_out = [torch.cuda.Event() for _ in range(nb)]     # codes of set b on the host
+        for b in range(nb):
+            ev_used[b].record(stream)
+            ev_out[b].record(stream)
+        ke = max(2, min(args.steps, 6))
 
-        def e2e_step():
-            dW.copy_(hW, non_blocking=True)
-            dUA.copy_(hUA, non_blocking=True)
-            dUB.copy_(hUB, non_blocking=True)
-            ds.copy_(hs, non_blocking=True)
-            q.run(dW, dUA, dUB, ds, spec.qmin, spec.qmax)
-            hcodes.copy_(q.codes, non_blocking=True)
-        e2e_step()
+        def e2e_step(k):
+            b = k % nb
+            dW_, dUA_, dUB_, ds_ = bufs[b]
+            h2d.wait_event(ev_used[b])
+            with torch.cuda.stream(h2d):
+                dW_.copy_(hW, non_blocking=True)
+                dUA_.copy_(hUA, non_blocking=True)
+                dUB_.copy_(hUB, non_blocking=True)
+                ds_.copy_(hs, non_blocking=True)
+            ev_in[b].record(h2d)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])          # set b's previous codes have left the device
+            qs[b].run(dW_, dUA_, dUB_, ds_, spec.qmin, spec.qmax, stream=stream)
+            ev_used[b].record(stream)
+            d2h.wait_event(ev_used[b])
+            with torch.cuda.stream(d2h):
+                hcodes[b].copy_(qs[b].codes, non_blocking=True)
+            ev_out[b].record(d2h)
+
+        for k in range(nb):
+            e2e_step(k)
+        torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
-        for _ in range(ke):
-            e2e_step()
+        h2d.wait_event(f0)
+        for k in range(ke):
+            e2e_step(k)
+        for b in range(nb):
+            stream.wait_event(ev_out[b])
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        for q_ in qs:
+            if q_.status() != 0:
+                raise RuntimeError(f"e2e solve status {q_.status()}")
         t_e2e = max_over_ranks(f0.elapsed_time(f1))
         e2e = {"value": world * ke * weights / (t_e2e / 1e3), "unit": "weights/s",
                "h2d_bytes_per_step": int(hW.numel() * es + hUA.numel() * es + hUB.numel() * es + hs.numel() * es),
-               "d2h_bytes_per_step": int(hcodes.numel()), "ms_per_step": t_e2e / ke}
+               "d2h_bytes_per_step": int(m * n), "ms_per_step": t_e2e / ke, "steps": ke,
+               "note": "pipelined: step k+1's host-to-device copies overlap step k's solve; every step's "
+                       "copies are inside the timed region"}
 
     block = None
     if rank == 0 and world == 1 and not args.no_block:

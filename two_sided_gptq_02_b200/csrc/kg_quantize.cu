@@ -325,42 +325,53 @@ static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
     return solve_range(a, s, mid, D1);
 }
 
-// Per host thread and device: the bulk stream and its events, created on first use and kept for
-// the life of the process.
-struct SchedPool {
-    int dev = -1;
+// Per host thread and device: a few bulk streams with their events, created on first use and kept
+// for the life of the process.  Calls take them in turn, so that solves in flight at the same time
+// on different caller streams (several layers at once) also run their bulk updates side by side;
+// two calls that share a slot only serialise their bulk work.
+struct SchedSlot {
     cudaStream_t bulk = nullptr;
     cudaEvent_t fork = nullptr;
     std::vector<cudaEvent_t> done;
 };
+struct SchedPool {
+    int dev = -1;
+    unsigned next = 0;
+    std::vector<SchedSlot> slots;
+};
+static constexpr int kSchedSlots = 8;
 static constexpr int kSchedDone = 64;
 
-static int sched_pool(SchedPool*& out) {
+static int sched_slot(SchedSlot*& out) {
     static thread_local std::vector<SchedPool> pools;
     int dev = 0;
     KG_CUDA_TRY(cudaGetDevice(&dev));
+    SchedPool* pool = nullptr;
     for (auto& p : pools)
-        if (p.dev == dev) {
-            out = &p;
-            return KG_OK;
+        if (p.dev == dev) pool = &p;
+    if (!pool) {
+        SchedPool p;
+        p.dev = dev;
+        p.slots.resize(kSchedSlots);
+        for (auto& sl : p.slots) {
+            KG_CUDA_TRY(cudaStreamCreateWithFlags(&sl.bulk, cudaStreamNonBlocking));
+            KG_CUDA_TRY(cudaEventCreateWithFlags(&sl.fork, cudaEventDisableTiming));
+            sl.done.resize(kSchedDone);
+            for (auto& e : sl.done) KG_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
         }
-    SchedPool p;
-    p.dev = dev;
-    KG_CUDA_TRY(cudaStreamCreateWithFlags(&p.bulk, cudaStreamNonBlocking));
-    KG_CUDA_TRY(cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming));
-    p.done.resize(kSchedDone);
-    for (auto& e : p.done) KG_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
-    pools.push_back(std::move(p));
-    out = &pools.back();
+        pools.push_back(std::move(p));
+        pool = &pools.back();
+    }
+    out = &pool->slots[pool->next++ % pool->slots.size()];
     return KG_OK;
 }
 
 template <typename Real>
 static int solve_all(const QArgs<Real>& a, int ndiag) {
-    SchedPool* pool = nullptr;
-    int rc = sched_pool(pool);
+    SchedSlot* slot = nullptr;
+    int rc = sched_slot(slot);
     if (rc) return rc;
-    Sched s{a.st, pool->bulk, pool->fork, pool->done.data(), (int)pool->done.size(), std::vector<int>(ndiag + 1, -1)};
+    Sched s{a.st, slot->bulk, slot->fork, slot->done.data(), (int)slot->done.size(), std::vector<int>(ndiag + 1, -1)};
     rc = solve_range(a, s, 0, ndiag);
     // join: the caller's stream waits for the last bulk update (also on the error path, so the
     // bulk stream never runs past the caller's view of the solve)
