@@ -258,6 +258,59 @@ def _cpu_baseline(spec, W, A, B, damp, budget_s=12.0):
                       f"{spec.m}x{spec.n} layer scales by (mn)^2 (extrapolated {t * (spec.m * spec.n / (mb * nb)) ** 2:.3g} s)"}
 
 
+# ---------------------------------------------------------------------------------------------- ranks
+class Replicas:
+    """The multi-GPU plumbing of the bench: one process per GPU, each an independent replica.
+
+    The solve does not shard (every layer is one sequential recursion over its anti-diagonals), so
+    each rank solves its own seeded layer and no data crosses between ranks. The only collectives
+    are the barriers around the timed region and one max-reduction of each rank's device time, so
+    that the job's time is that of its slowest rank. `backend` is "nccl" on GPUs and "gloo" for the
+    same logic on host cores.
+    """
+
+    SEED_STRIDE = 7919
+
+    def __init__(self, rank: int, world: int, backend: str = "nccl", device=None, timeout_s: float = 180.0):
+        import torch
+        import torch.distributed as dist
+        self.rank, self.world, self.backend = rank, world, backend
+        self.device = device if device is not None else torch.device("cpu")
+        self._dist = dist
+        if world > 1 and not dist.is_initialized():
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self) -> None:
+        if self.world == 1:
+            return
+        if self.backend == "nccl":
+            self._dist.barrier(device_ids=[self.device.index])
+        else:
+            self._dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def replica_spec(self, base):
+        """This rank's layer: the workload's shape with a seed of its own."""
+        from synth_inputs.layers import LayerSpec
+        return LayerSpec(**{**base.__dict__, "seed": base.seed + self.SEED_STRIDE * self.rank})
+
+    def job_throughput(self, units_per_rank: float, seconds_max: float) -> float:
+        """Whole-job units/s: every rank's units over the slowest rank's time."""
+        return self.world * units_per_rank / seconds_max
+
+    def close(self) -> None:
+        if self.world > 1 and self._dist.is_initialized():
+            self._dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -291,29 +344,16 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import two_sided_gptq_02_b200 as kg
-    from synth_inputs.layers import LayerSpec, layer_inputs, workload
+    from synth_inputs.layers import layer_inputs, workload
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    ranks = Replicas(rank, world, "nccl", dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    base = workload(args.workload)[0]
-    spec = LayerSpec(**{**base.__dict__, "seed": base.seed + 7919 * rank})
+    spec = ranks.replica_spec(workload(args.workload)[0])
     dt = torch.float32 if args.dtype == "f32" else torch.float64
     W, A, B = layer_inputs(spec, device=dev)
     UA, UB, UA32, UB32 = kg.kron_gptq_prepare(A, B, args.damp)
@@ -354,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
     ms_max = max_over_ranks(ms)
     clocks = clk.summary()
     weights = spec.m * spec.n
-    value = world * args.steps * weights / (ms_max / 1e3)
+    value = ranks.job_throughput(args.steps * weights, ms_max / 1e3)
     ms_per_step = ms_max / args.steps
 
     # ---- per-kernel durations (separate pass with event timing of every launch)
@@ -479,7 +519,7 @@ def run_ours(args, rank, world, local_rank):
             if q_.status() != 0:
                 raise RuntimeError(f"e2e solve status {q_.status()}")
         t_e2e = max_over_ranks(f0.elapsed_time(f1))
-        e2e = {"value": world * ke * weights / (t_e2e / 1e3), "unit": "weights/s",
+        e2e = {"value": ranks.job_throughput(ke * weights, t_e2e / 1e3), "unit": "weights/s",
                "h2d_bytes_per_step": int(hW.numel() * es + hUA.numel() * es + hUB.numel() * es + hs.numel() * es),
                "d2h_bytes_per_step": int(m * n), "ms_per_step": t_e2e / ke, "steps": ke,
                "note": "pipelined: step k+1's host-to-device copies overlap step k's solve; every step's "
@@ -509,8 +549,7 @@ def run_ours(args, rank, world, local_rank):
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
                           "source": peak_src}}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
