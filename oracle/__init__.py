@@ -22,6 +22,14 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
                   loss identity, error bound, certificate.
   quantize_onesided  pinned: the vectorized form with B=I, RTN when A is diagonal.
   loss            pinned: closed forms (sum E^2) and numpy einsum of the definition.
+  quantize_rc     pinned: literal vectorized form with a per-entry step (4x4, 6x5, ...),
+                  A=B=I reduces to per-entry rounding, alpha=1 / beta=s equals
+                  quantize_naive on an unclipped grid, certificate, |E| <= gamma/2 for the
+                  WaterKron steps.
+  waterkron_scales  the formula itself (one line); pinned through the |E| <= gamma/2 bound
+                  and the high-rate distortion mn gamma^2 / 12.
+  code_entropy_bits pinned: closed forms (uniform over 2^k symbols gives k bits, a constant
+                  gives 0, a two-point law gives its binary entropy).
 """
 from __future__ import annotations
 
@@ -67,6 +75,8 @@ def _load():
             lib.ora_quantize_naive.argtypes = [P, I64, I64, P, P, P, ctypes.c_int, ctypes.c_int, P,
                                                ctypes.c_double, P, P, P, P, P]
             lib.ora_quantize_naive.restype = I64
+            lib.ora_quantize_rc.argtypes = [P, I64, I64, P, P, P, P, P, ctypes.c_double, P, P, P, P, P]
+            lib.ora_quantize_rc.restype = I64
             lib.ora_quantize_onesided.argtypes = [P, I64, I64, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
             lib.ora_quantize_onesided.restype = None
             lib.ora_rtn.argtypes = [P, I64, I64, P, ctypes.c_int, ctypes.c_int, P, P]
@@ -132,6 +142,54 @@ def quantize_naive(W, UA, UB, s, qmin: int, qmax: int, *, forced=None, tol: floa
     return dict(codes=codes, V=V, E=E, t=t, boundary=bflag.astype(bool), n_boundary=int(nb))
 
 
+NOT_FORCED_64 = -(2 ** 63)
+
+
+def quantize_rc(W, UA, UB, alpha, beta, *, forced=None, tol: float = 1e-9):
+    """Two-sided GPTQ by definition on the alphabet V = beta alpha^T (.) Z, Z unbounded
+    ("WaterKron and FlipFlop Hessian", Section 2.1).  Returns dict(codes (int64), V, E, t,
+    boundary, n_boundary); ``forced`` uses NOT_FORCED_64 for entries left to the rounding."""
+    W, UA, UB, alpha, beta = _f64(W), _f64(UA), _f64(UB), _f64(alpha), _f64(beta)
+    m, n = W.shape
+    assert UA.shape == (n, n) and UB.shape == (m, m) and alpha.shape == (n,) and beta.shape == (m,)
+    codes = np.zeros((m, n), dtype=np.int64)
+    V = np.zeros((m, n), dtype=np.float64)
+    E = np.zeros((m, n), dtype=np.float64)
+    t = np.zeros((m, n), dtype=np.float64)
+    bflag = np.zeros((m, n), dtype=np.uint8)
+    f = None
+    if forced is not None:
+        f = np.ascontiguousarray(forced, dtype=np.int64)
+        assert f.shape == (m, n)
+    nb = _load().ora_quantize_rc(_ptr(W), m, n, _ptr(UA), _ptr(UB), _ptr(alpha), _ptr(beta), _ptr(f),
+                                 float(tol), _ptr(codes), _ptr(V), _ptr(E), _ptr(t), _ptr(bflag))
+    if nb < 0:
+        raise MemoryError("oracle quantize_rc: allocation failed")
+    return dict(codes=codes, V=V, E=E, t=t, boundary=bflag.astype(bool), n_boundary=int(nb))
+
+
+def waterkron_scales(UA, UB, gamma: float):
+    """WaterKron steps ("WaterKron and FlipFlop Hessian", Section 3): alpha_j proportional to
+    1 / L^(A)_jj = U_A[j,j] and beta_i proportional to U_B[i,i].  One knob gamma > 0 sets
+    both constants (alpha = sqrt(gamma) diag U_A, beta = sqrt(gamma) diag U_B), so that the
+    step of entry (i,j) is gamma U_B[i,i] U_A[j,j] and every error E_ij = (x - Q)/(U_B[i,i]
+    U_A[j,j]) lies in [-gamma/2, gamma/2]."""
+    r = np.sqrt(float(gamma))
+    return r * np.diag(_f64(UA)).copy(), r * np.diag(_f64(UB)).copy()
+
+
+def code_entropy_bits(Z) -> float:
+    """Empirical (plug-in) entropy of the integer entries of Z in bits per entry: the
+    memory cost of Z under a good entropy coder ("WaterKron and FlipFlop Hessian",
+    Section 2.1).  H = -sum_z p_z log2 p_z with p_z the frequency of value z."""
+    Z = np.asarray(Z).reshape(-1)
+    if Z.size == 0:
+        return 0.0
+    _, counts = np.unique(Z, return_counts=True)
+    p = counts.astype(np.float64) / Z.size
+    return float(-(p * np.log2(p)).sum())
+
+
 def quantize_onesided(W, U, S, qmin: int, qmax: int):
     """Standard GPTQ with per-entry scale S (m x n).  Returns dict(codes, V, E)."""
     W, U, S = _f64(W), _f64(U), _f64(S)
@@ -161,8 +219,10 @@ def loss(W, V, Ad, Bd) -> float:
 
 from .literal import (  # noqa: E402,F401
     certificate,
+    certificate_rc,
     damped,
     literal_vec,
+    literal_vec_entry,
     prepare_lapack,
 )
 from .parity import compare_with_oracle  # noqa: E402,F401

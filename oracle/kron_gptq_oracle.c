@@ -199,6 +199,59 @@ int64_t ora_quantize_naive(const double* W, int64_t m, int64_t n,
 }
 
 /* ------------------------------------------------------------------------------------
+ * The same algorithm on the row- and column-scaled alphabet with unbounded integers
+ * [WK Sec. 2.1: V = beta alpha^T (.) Z with Z integer and not clipped; the scales are
+ * chosen up front and handed to the algorithm].  Entry (i,j) has grid step
+ * s_ij = beta_i * alpha_j:
+ *     x = W~[i,j];  z = rint(x / s_ij);  Q = s_ij z;  e = (x - Q) / (U_B[i,i] U_A[j,j]);
+ * followed by the same bottom-right update as ora_quantize_naive.  Codes are int64.
+ * forced (nullable): a code other than INT64_MIN replaces the decision at that entry.
+ * Returns the number of boundary entries (|x/s_ij - half-integer| < tol).
+ * ------------------------------------------------------------------------------------ */
+int64_t ora_quantize_rc(const double* W, int64_t m, int64_t n,
+                        const double* UA, const double* UB, const double* alpha, const double* beta,
+                        const int64_t* forced, double tol,
+                        int64_t* codes, double* V, double* E, double* tpre, uint8_t* bflag)
+{
+    double* Wt = (double*)malloc(sizeof(double) * (size_t)(m * n));
+    if (!Wt) return -1;
+    memcpy(Wt, W, sizeof(double) * (size_t)(m * n));
+    int64_t nb = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        for (int64_t i = 0; i < m; ++i) {
+            const int64_t p = i * n + j;
+            const double x = Wt[p];
+            const double sij = beta[i] * alpha[j];
+            const double t = x / sij;
+            double z;
+            if (forced && forced[p] != INT64_MIN) z = (double)forced[p];
+            else z = rint(t);
+            const double f = floor(t);
+            const int b = fabs(t - (f + 0.5)) < tol;
+            nb += b;
+            if (bflag) bflag[p] = (uint8_t)b;
+            if (tpre) tpre[p] = t;
+            const double q = sij * z;
+            const double e = (x - q) / (UB[i * m + i] * UA[j * n + j]);
+            codes[p] = (int64_t)z;
+            V[p] = q;
+            if (E) E[p] = e;
+            for (int64_t ip = i; ip < m; ++ip) {
+                const double be = UB[i * m + ip] * e;
+                if (be == 0.0) continue;
+                double* row = Wt + ip * n;
+                for (int64_t jp = j; jp < n; ++jp) {
+                    if (ip == i && jp == j) continue;
+                    row[jp] -= be * UA[j * n + jp];
+                }
+            }
+        }
+    }
+    free(Wt);
+    return nb;
+}
+
+/* ------------------------------------------------------------------------------------
  * Standard one-sided GPTQ [FK Sec. 2.2, "Algorithm 1"; WK Sec. 2.2]: columns in order,
  * all rows of a column rounded at once, error fed forward along the row through the
  * upper Cholesky factor U of A_d^{-1}.  The scale is given per entry (S, m x n) so that

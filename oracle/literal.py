@@ -7,7 +7,8 @@
 * ``prepare_lapack``: the same four prepare steps as the C oracle (damp, Cholesky,
   inverse, upper Cholesky of the inverse) with numpy's LAPACK routines as the steps;
   used where the textbook C loops would take minutes.
-* ``certificate``: a check of a solver's output that holds at any size.  The
+* ``literal_vec_entry``: the same with a step per coordinate and unclipped integers.
+* ``certificate`` / ``certificate_rc``: a check of a solver's output that holds at any size.  The
   recurrences of two-sided GPTQ imply V - W = -U_B^T E U_A exactly (each update adds a
   column of kron(U_A,U_B)^T times the scaled error), and every code is the rounding of
   the value W~ = V + E * (u_B u_A^T) the entry had when it was visited (u = diag U).
@@ -64,6 +65,66 @@ def literal_vec(W, Ad, Bd, s, qmin: int, qmax: int, forced=None):
         w[p + 1:] -= e[p] * K[p, p + 1:]
     unvec = lambda v: v.reshape(n, m).T.copy()
     return dict(codes=unvec(c).astype(np.int32), V=unvec(q), E=unvec(e), K=K)
+
+
+def literal_vec_entry(W, Ad, Bd, S):
+    """1-D GPTQ on w = vecop(W) with Gram kron(Ad, Bd) and a step per coordinate
+    (S, m x n), integers not clipped ("WaterKron and FlipFlop Hessian", Sections 2.1 and 3:
+    alpha-hat = alpha (x) beta on the vectorized problem)."""
+    W = np.asarray(W, dtype=np.float64)
+    m, n = W.shape
+    H = np.kron(np.asarray(Ad, dtype=np.float64), np.asarray(Bd, dtype=np.float64))
+    Hi = np.linalg.inv(H)
+    Hi = 0.5 * (Hi + Hi.T)
+    K = np.linalg.cholesky(Hi).T
+    w = W.T.reshape(-1).copy()
+    svec = np.asarray(S, dtype=np.float64).T.reshape(-1)
+    N = m * n
+    c = np.zeros(N, dtype=np.int64)
+    q = np.zeros(N)
+    e = np.zeros(N)
+    for p in range(N):
+        x = w[p]
+        c[p] = np.rint(x / svec[p])
+        q[p] = svec[p] * c[p]
+        e[p] = (x - q[p]) / K[p, p]
+        w[p + 1:] -= e[p] * K[p, p + 1:]
+    unvec = lambda v: v.reshape(n, m).T.copy()
+    return dict(codes=unvec(c), V=unvec(q), E=unvec(e), K=K)
+
+
+def certificate_rc(W, UA, UB, alpha, beta, codes, V, E, rows=None, tol: float = 1e-9):
+    """The certificate for the row- and column-scaled alphabet: (1) V - W + U_B^T E U_A = 0,
+    (2) codes = rint(W~ / (beta_i alpha_j)), (3) |W~ - V| <= step / 2, with
+    W~ = V + E * (u_B u_A^T)."""
+    W = np.asarray(W, dtype=np.float64)
+    UA = np.asarray(UA, dtype=np.float64)
+    UB = np.asarray(UB, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    E = np.asarray(E, dtype=np.float64)
+    alpha = np.asarray(alpha, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    codes = np.asarray(codes)
+    m, n = W.shape
+    if rows is None:
+        rows = np.arange(m)
+        corr = UB.T @ E @ UA
+    else:
+        rows = np.asarray(rows)
+        corr = np.stack([(UB[: i + 1, i] @ E[: i + 1, :]) @ UA for i in rows])
+    resid = V[rows] - W[rows] + corr
+    scale = max(np.abs(W[rows]).max(), 1e-300)
+    uB = np.diag(UB)[rows]
+    uA = np.diag(UA)
+    Wt = V[rows] + E[rows] * (uB[:, None] * uA[None, :])
+    step = beta[rows, None] * alpha[None, :]
+    t = Wt / step
+    f = np.floor(t)
+    tie = np.abs(t - (f + 0.5)) < tol
+    mism = (np.rint(t) != codes[rows]) & ~tie
+    half = np.abs(Wt - V[rows]) > (0.5 + tol) * step
+    return dict(resid_abs=float(np.abs(resid).max()), resid_rel=float(np.abs(resid).max() / scale),
+                code_mismatch=int(mism.sum()), halfstep_violations=int(half.sum()), rows=len(rows))
 
 
 def certificate(W, UA, UB, s, qmin: int, qmax: int, codes, V, E, rows=None, tol: float = 1e-9):

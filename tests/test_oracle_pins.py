@@ -306,3 +306,138 @@ def test_generator_leading_block_is_consistent():
     assert np.array_equal(W[:16, :16].numpy(), Wl.numpy())
     np.testing.assert_allclose(A[:16, :16].numpy(), Al.numpy(), rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(B[:16, :16].numpy(), Bl.numpy(), rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- row- and column-scaled alphabet
+# "WaterKron and FlipFlop Hessian", Section 2.1: V = beta alpha^T (.) Z with Z integer and not
+# clipped; Section 3: the WaterKron steps alpha_j ~ U_A[j,j], beta_i ~ U_B[i,i].
+
+def _rc_case(m, n, seed, gamma=None, scale_w=1.0):
+    f = _factors(m, n, seed)
+    W = f["W"] * scale_w
+    if gamma is None:
+        rng = np.random.default_rng(seed)
+        alpha = 0.05 * np.exp(0.5 * rng.standard_normal(n))
+        beta = np.exp(0.5 * rng.standard_normal(m))
+    else:
+        alpha, beta = oracle.waterkron_scales(f["UA"], f["UB"], gamma)
+    return f, W, alpha, beta
+
+
+@pytest.mark.parametrize("m,n,seed,gamma", [(4, 4, 0, None), (6, 5, 1, None), (5, 7, 2, 0.7), (3, 8, 3, 0.2),
+                                            (8, 3, 4, 1.5)])
+def test_rc_equals_literal_vectorized(m, n, seed, gamma):
+    f, W, alpha, beta = _rc_case(m, n, seed, gamma)
+    r = oracle.quantize_rc(W, f["UA"], f["UB"], alpha, beta)
+    lit = oracle.literal_vec_entry(W, f["Ad"], f["Bd"], beta[:, None] * alpha[None, :])
+    assert r["n_boundary"] == 0
+    np.testing.assert_array_equal(r["codes"], lit["codes"])
+    np.testing.assert_allclose(r["V"], lit["V"], rtol=0, atol=0)
+    np.testing.assert_allclose(r["E"], lit["E"], rtol=1e-9, atol=1e-12)
+    assert np.abs(r["codes"]).max() > 0
+
+
+def test_rc_identity_factors_is_entrywise_rounding():
+    f, W, alpha, beta = _rc_case(12, 10, 71, scale_w=40.0)
+    step = beta[:, None] * alpha[None, :]
+    r = oracle.quantize_rc(W, np.eye(10), np.eye(12), alpha, beta)
+    np.testing.assert_array_equal(r["codes"], np.rint(W / step).astype(np.int64))
+    np.testing.assert_array_equal(r["V"], step * np.rint(W / step))
+    # unbounded: codes far outside any clipped grid survive
+    assert np.abs(r["codes"]).max() > 127
+
+
+def test_rc_with_unit_columns_is_the_row_scaled_algorithm():
+    # alpha = 1 and beta = s: the row-scaled algorithm on a grid too wide to clip
+    f = _factors(14, 11, 72)
+    big = 2 ** 30
+    r = oracle.quantize_rc(f["W"], f["UA"], f["UB"], np.ones(11), f["s"] * 0.05)
+    ref = oracle.quantize_naive(f["W"], f["UA"], f["UB"], f["s"] * 0.05, -big, big - 1)
+    np.testing.assert_array_equal(r["codes"], ref["codes"].astype(np.int64))
+    np.testing.assert_array_equal(r["V"], ref["V"])
+    np.testing.assert_array_equal(r["E"], ref["E"])
+
+
+def test_waterkron_error_bound_certificate_and_loss():
+    gamma = 0.4
+    f, W, alpha, beta = _rc_case(20, 16, 73, gamma)
+    r = oracle.quantize_rc(W, f["UA"], f["UB"], alpha, beta)
+    # with steps gamma U_B[i,i] U_A[j,j] every error lies in [-gamma/2, gamma/2]
+    assert np.abs(r["E"]).max() <= 0.5 * gamma * (1 + 1e-12)
+    c = oracle.certificate_rc(W, f["UA"], f["UB"], alpha, beta, r["codes"], r["V"], r["E"])
+    assert c["resid_rel"] < 1e-12 and c["code_mismatch"] == 0 and c["halfstep_violations"] == 0
+    # the proxy loss is sum E^2 for any alphabet (V - W = -U_B^T E U_A)
+    lt = oracle.loss(W, r["V"], f["Ad"], f["Bd"])
+    assert abs(lt - np.sum(r["E"] ** 2)) < 1e-10 * lt
+    # a corrupted code breaks the certificate
+    bad = r["codes"].copy()
+    bad[3, 5] += 1
+    c2 = oracle.certificate_rc(W, f["UA"], f["UB"], alpha, beta, bad, r["V"], r["E"])
+    assert c2["code_mismatch"] == 1
+
+
+def test_waterkron_high_rate_distortion():
+    # high rate: the transformed errors are uniform on [-gamma/2, gamma/2], so the mean of E^2
+    # is gamma^2 / 12 ("WaterKron and FlipFlop Hessian", Appendix C.2, the limit gamma -> 0)
+    gamma = 0.02
+    f, W, alpha, beta = _rc_case(64, 64, 74, gamma)
+    r = oracle.quantize_rc(W, f["UA"], f["UB"], alpha, beta)
+    ratio = np.mean(r["E"] ** 2) / (gamma ** 2 / 12)
+    assert abs(ratio - 1.0) < 0.05, ratio
+    # halving gamma adds about one bit per entry to the empirical entropy of Z
+    alpha2, beta2 = oracle.waterkron_scales(f["UA"], f["UB"], gamma / 2)
+    r2 = oracle.quantize_rc(W, f["UA"], f["UB"], alpha2, beta2)
+    dh = oracle.code_entropy_bits(r2["codes"]) - oracle.code_entropy_bits(r["codes"])
+    assert abs(dh - 1.0) < 0.1, dh
+
+
+def test_code_entropy_closed_forms():
+    assert oracle.code_entropy_bits(np.full((7, 9), -3)) == 0.0
+    z = np.tile(np.array([-2, 0, 5, 1000]), 25)
+    assert oracle.code_entropy_bits(z) == pytest.approx(2.0, abs=1e-15)
+    z = np.array([0] * 300 + [-7] * 100)
+    h = -(0.75 * np.log2(0.75) + 0.25 * np.log2(0.25))
+    assert oracle.code_entropy_bits(z) == pytest.approx(h, abs=1e-15)
+    assert oracle.code_entropy_bits(np.arange(256)) == pytest.approx(8.0, abs=1e-12)
+
+
+def _rc_py(W, UA, UB, alpha, beta, mutation=None):
+    """A pure-Python copy of the scaled-alphabet loop with one planted mistake."""
+    m, n = W.shape
+    Wt = W.copy()
+    codes = np.zeros((m, n), dtype=np.int64)
+    V = np.zeros((m, n))
+    E = np.zeros((m, n))
+    for j in range(n):
+        for i in range(m):
+            x = Wt[i, j]
+            sij = beta[i] * alpha[j] if mutation != "row_step_only" else beta[i]
+            z = np.rint(x / sij)
+            if mutation == "clip_int8":
+                z = min(max(z, -128), 127)
+            q = sij * z
+            e = (x - q) / (UB[i, i] * UA[j, j])
+            if mutation == "error_in_grid_units":
+                e = (x - q) / sij
+            codes[i, j], V[i, j], E[i, j] = z, q, e
+            for ip in range(i, m):
+                for jp in range(j, n):
+                    if ip == i and jp == j:
+                        continue
+                    Wt[ip, jp] -= UB[i, ip] * e * UA[j, jp]
+    return codes, V, E
+
+
+@pytest.mark.parametrize("mutation", ["row_step_only", "clip_int8", "error_in_grid_units"])
+def test_planted_mistakes_fail_an_rc_pin(mutation):
+    f, W, alpha, beta = _rc_case(6, 5, 75)
+    W = W * 40.0                       # codes beyond the int8 range
+    args = (W, f["UA"], f["UB"], alpha, beta)
+    c0, V0, E0 = _rc_py(*args)
+    ref = oracle.quantize_rc(*args)
+    np.testing.assert_array_equal(c0, ref["codes"])       # the unmutated copy agrees
+    c, V, E = _rc_py(*args, mutation=mutation)
+    lit = oracle.literal_vec_entry(W, f["Ad"], f["Bd"], beta[:, None] * alpha[None, :])
+    cert = oracle.certificate_rc(*args, c, V, E)
+    caught = (not np.array_equal(c, lit["codes"])) or cert["resid_rel"] > 1e-9 or cert["code_mismatch"] > 0
+    assert caught, mutation
