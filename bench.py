@@ -49,6 +49,8 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-block", action="store_true")
+    ap.add_argument("--no-waterkron", action="store_true")
+    ap.add_argument("--gamma", type=float, default=0.02, help="WaterKron step knob for the scaled-alphabet line")
     return ap.parse_args()
 
 
@@ -188,6 +190,37 @@ def _block_seconds(kg, torch, damp, reps=3):
             "dtype": "f32", "bits": 3, "seconds_per_block_one_stream": seq,
             "seconds_per_block_seven_streams": con, "weights_per_s_seven_streams": weights / con, "reps": reps,
             "note": "inputs on the device; each layer its own seeded W, A, B (N=4096 rows); median of reps"}
+
+
+def _waterkron(kg, torch, spec, Wd, UAd, UBd, gamma, steps, solve_ms, roofline_ms):
+    """The same layer on the WaterKron alphabet (row and column steps, unclipped int32 codes):
+    device time per solve with inputs resident, the rate (entropy of Z) and the distortion against
+    the high-rate value gamma^2 / 12 per entry."""
+    stream = torch.cuda.current_stream()
+    alpha, beta = kg.kron_gptq_waterkron_scales(UAd, UBd, gamma)
+    q = kg.RcQuantizer(spec.m, spec.n, Wd.dtype, Wd.device, want_E=True)
+    for _ in range(2):
+        q.run(Wd, UAd, UBd, alpha, beta)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        q.run(Wd, UAd, UBd, alpha, beta)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = q.status()
+    if st != 0:
+        raise kg.KGError(st, "waterkron solve")
+    ms = e0.elapsed_time(e1) / steps
+    bits = kg.kron_gptq_code_entropy(q.Z)
+    mse = float((q.E.double() ** 2).mean().item())
+    return {"gamma": gamma, "ms_per_solve": ms, "weights_per_s": spec.m * spec.n / (ms / 1e3),
+            "overhead_vs_row_scaled": ms / solve_ms - 1.0,
+            "solve_roofline_frac": roofline_ms / ms,
+            "entropy_bits_per_weight": bits, "max_abs_code": int(q.Z.abs().max().item()),
+            "mean_E2_over_gamma2_12": mse / (gamma ** 2 / 12.0), "steps": steps,
+            "note": "kron_gptq_quantize_rc with kron_gptq_waterkron_scales on the same layer and dtype; "
+                    "inputs resident; the step rescaling and the V, E rescaling are inside the time"}
 
 
 def _traffic(kernel: str, units_per_launch: float):
@@ -529,6 +562,11 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_block:
         block = _block_seconds(kg, torch, args.damp)
 
+    waterkron = None
+    if rank == 0 and world == 1 and not args.no_waterkron:
+        waterkron = _waterkron(kg, torch, spec, Wd, UAd, UBd, args.gamma, max(3, min(args.steps, 10)), ms_per_step,
+                               solve["roofline_ms"])
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(spec, W, A, B, args.damp)
@@ -545,7 +583,7 @@ def run_ours(args, rank, world, local_rank):
                                  f"{(bytes_compulsory + 3 * m * n * es) / 1e6:.0f} MB)"},
                 "roofline": rl, "roofline_other": rl_other, "solve_roofline": solve, "kernel_breakdown": breakdown,
                 "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
-                "block": block,
+                "block": block, "waterkron": waterkron,
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
                           "source": peak_src}}
         print(json.dumps(line), flush=True)

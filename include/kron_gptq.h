@@ -53,7 +53,9 @@ typedef enum kg_status {
     KG_ERR_WORKSPACE = -4,    /* workspace smaller than *_workspace_size() */
     KG_ERR_NOT_PD = -5,       /* (device) a Cholesky pivot was not positive */
     KG_ERR_NONFINITE = -6,    /* (device) NaN/Inf in W, in the scales or in a factor diagonal */
-    KG_ERR_TIMEOUT = -7       /* (device) a bounded device-side wait ran out */
+    KG_ERR_TIMEOUT = -7,      /* (device) a bounded device-side wait ran out */
+    KG_ERR_RANGE = -8         /* (device) an unclipped code reached the representable bound, or
+                                 the codes span more values than the entropy workspace has bins */
 } kg_status;
 
 typedef enum kg_dtype {
@@ -186,6 +188,65 @@ KG_API int kron_gptq_quantize_noalloc(const void* W, int64_t m, int64_t n, int d
                                       const void* U_A, const void* U_B, kg_grid grid,
                                       int8_t* out_codes, void* out_V, void* out_E,
                                       int* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_quantize_rc -- two-sided GPTQ on the row- and column-scaled alphabet with unclipped
+ *   integers ("WaterKron and FlipFlop Hessian", Section 2.1: V = beta alpha^T (.) Z, Z integer
+ *   and not clipped, the scales chosen up front and handed to the algorithm).  For entry (i,j)
+ *   with current value x and step s_ij = beta_i alpha_j:
+ *       z = rint(x / s_ij),  Q = s_ij z,  E_ij = (x - Q) / (U_B[i,i] U_A[j,j]),
+ *   then the same update as kron_gptq_quantize.  Computed by the same solve on the rescaled
+ *   problem W (/) (beta alpha^T) with factors D_alpha U_A D_alpha^-1, D_beta U_B D_beta^-1 (the
+ *   two are the same algorithm: dividing every update by the target's step turns one into the
+ *   other), then V = s (.) Z and E = s (.) E'.
+ * Arguments:
+ *   W, U_A, U_B, dtype, m, n   as kron_gptq_quantize.
+ *   alpha     device, n entries of dtype, each finite and > 0 (column steps).
+ *   beta      device, m entries of dtype, each finite and > 0 (row steps).
+ *   out_Z     device, m x n int32 codes.
+ *   out_V     device, m x n, dtype: V = beta_i alpha_j Z_ij.
+ *   out_E     optional device, m x n, dtype (NULL to skip): V - W = -U_B^T E U_A.
+ *   ws        kron_gptq_quantize_rc_workspace_size(m, n, dtype) bytes, 256-byte aligned; its
+ *             first 256 bytes are the status word (kron_gptq_sync_status).
+ * The codes are unclipped up to |Z| < 2^22 in fp32 (where fp32 still holds every integer of the
+ * step) and |Z| < 2^30 in fp64; a code at that bound raises KG_ERR_RANGE.
+ * m == 0 or n == 0 is a no-op returning KG_OK.
+ * Device errors: KG_ERR_NONFINITE (NaN/Inf in W, a step not finite and > 0, a factor diagonal
+ *   not > 0), KG_ERR_RANGE, KG_ERR_TIMEOUT.
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_quantize_rc_workspace_size(int64_t m, int64_t n, int dtype);
+KG_API int kron_gptq_quantize_rc(const void* W, int64_t m, int64_t n, int dtype,
+                                 const void* U_A, const void* U_B, const void* alpha, const void* beta,
+                                 int32_t* out_Z, void* out_V, void* out_E,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_waterkron_scales -- the WaterKron steps ("WaterKron and FlipFlop Hessian",
+ *   Section 3: alpha_j proportional to 1/L^(A)_jj and beta_i to 1/L^(B)_ii, where L is the
+ *   reverse Cholesky factor, so 1/L^(A)_jj = U_A[j,j]).  One knob gamma > 0 sets both constants:
+ *       alpha_j = sqrt(gamma) U_A[j,j],   beta_i = sqrt(gamma) U_B[i,i],
+ *   so the step of entry (i,j) is gamma U_B[i,i] U_A[j,j] and every error E_ij of
+ *   kron_gptq_quantize_rc lies in [-gamma/2, gamma/2].
+ * Arguments: U_A (n x n), U_B (m x m) device factors of dtype; alpha (n), beta (m) device
+ *   outputs of dtype.  gamma must be finite and > 0 (else KG_ERR_ARG).
+ * --------------------------------------------------------------------------------------- */
+KG_API int kron_gptq_waterkron_scales(const void* U_A, int64_t n, const void* U_B, int64_t m, int dtype,
+                                      double gamma, void* alpha, void* beta, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_code_entropy -- empirical entropy of integer codes in bits per entry, the memory
+ *   cost of Z under a good entropy coder ("WaterKron and FlipFlop Hessian", Section 2.1):
+ *       H = -sum_z (c_z / N) log2(c_z / N),  c_z = number of entries equal to z.
+ * Arguments:
+ *   Z         device, count int32 codes (count < 2^32).
+ *   out_bits  device, one double (written in stream order; NaN when the range does not fit).
+ *   ws        kron_gptq_code_entropy_workspace_size(max_bins) bytes, 256-byte aligned: room for
+ *             max_bins distinct values between min(Z) and max(Z); status word first.
+ * Device errors: KG_ERR_RANGE when max(Z) - min(Z) + 1 exceeds the workspace's bins.
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_code_entropy_workspace_size(int64_t max_bins);
+KG_API int kron_gptq_code_entropy(const int32_t* Z, int64_t count, double* out_bits,
+                                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Diagnostics (tracing).  The library counts every kernel launch by kind:

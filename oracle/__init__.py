@@ -225,4 +225,4 @@ from .literal import (  # noqa: E402,F401
     literal_vec_entry,
     prepare_lapack,
 )
-from .parity import compare_with_oracle  # noqa: E402,F401
+from .parity import compare_with_oracle, compare_with_oracle_rc  # noqa: E402,F401

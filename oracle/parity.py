@@ -41,3 +41,30 @@ def compare_with_oracle(codes, W, UA, UB, s, qmin: int, qmax: int, *, tol: float
         for i, j in first:
             forced[i, j] = codes[i, j]
             flips.append((int(i), int(j), float(r["t"][i, j])))
+
+
+def compare_with_oracle_rc(codes, W, UA, UB, alpha, beta, *, tol: float = 1e-9, max_flips: int = 64):
+    """The same rule for the row- and column-scaled alphabet (oracle ``quantize_rc``)."""
+    from . import NOT_FORCED_64, quantize_rc
+    codes = np.asarray(codes).astype(np.int64)
+    m, n = codes.shape
+    forced = np.full((m, n), NOT_FORCED_64, dtype=np.int64)
+    flips = []
+    ii, jj = np.meshgrid(np.arange(m), np.arange(n), indexing="ij")
+    while True:
+        r = quantize_rc(W, UA, UB, alpha, beta, forced=forced, tol=tol)
+        diff = r["codes"] != codes
+        if not diff.any():
+            return dict(ok=True, flips=flips, oracle=r, mismatches=0)
+        d = np.where(diff, ii + jj, np.iinfo(np.int64).max)
+        dmin = d.min()
+        first = np.argwhere(d == dmin)
+        bad = [(int(i), int(j)) for i, j in first if not r["boundary"][i, j]]
+        if bad or len(flips) + len(first) > max_flips:
+            i, j = bad[0] if bad else tuple(first[0])
+            return dict(ok=False, flips=flips, oracle=r, mismatches=int(diff.sum()),
+                        first=(int(i), int(j)), t=float(r["t"][i, j]),
+                        oracle_code=int(r["codes"][i, j]), candidate_code=int(codes[i, j]))
+        for i, j in first:
+            forced[i, j] = codes[i, j]
+            flips.append((int(i), int(j), float(r["t"][i, j])))

@@ -11,6 +11,10 @@ Public functions mirror the C names:
     kron_gptq_quantize(W, U_A, U_B, ...)   -> codes (int8), V, E
     kron_gptq_loss(W, V, A, B, damp)       -> float
     kron_gptq_row_scales(W, qmax)          -> per-row scales
+    kron_gptq_quantize_rc(W, U_A, U_B, alpha, beta) -> Z (int32), V, E  (row- and column-scaled
+                                              alphabet, unclipped codes)
+    kron_gptq_waterkron_scales(U_A, U_B, gamma)     -> alpha, beta (WaterKron steps)
+    kron_gptq_code_entropy(Z)                       -> bits per entry
     kron_gptq_sync_status(ws, stream)      -> device status word
 """
 from __future__ import annotations
@@ -20,6 +24,7 @@ from ._lib import (  # noqa: F401
     KG_F64,
     KGError,
     Quantizer,
+    RcQuantizer,
     PROFILE_KINDS,
     kron_gptq_loss,
     kron_gptq_profile_enable,
@@ -27,6 +32,9 @@ from ._lib import (  # noqa: F401
     kron_gptq_prepare,
     kron_gptq_quantize,
     kron_gptq_quantize_noalloc,
+    kron_gptq_quantize_rc,
+    kron_gptq_code_entropy,
+    kron_gptq_waterkron_scales,
     kron_gptq_row_scales,
     kron_gptq_status_string,
     kron_gptq_sync_status,

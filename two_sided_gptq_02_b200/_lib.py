@@ -11,7 +11,7 @@ KG_F32 = 1
 KG_F64 = 2
 _ERRORS = {
     -1: "KG_ERR_ARG", -2: "KG_ERR_UNSUPPORTED", -3: "KG_ERR_CUDA", -4: "KG_ERR_WORKSPACE",
-    -5: "KG_ERR_NOT_PD", -6: "KG_ERR_NONFINITE", -7: "KG_ERR_TIMEOUT",
+    -5: "KG_ERR_NOT_PD", -6: "KG_ERR_NONFINITE", -7: "KG_ERR_TIMEOUT", -8: "KG_ERR_RANGE",
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +67,16 @@ def load_library():
         L.kron_gptq_sync_status.restype = I
         L.kron_gptq_quantize_noalloc.argtypes = [P, I64, I64, I, P, P, _Grid, P, P, P, P, P]
         L.kron_gptq_quantize_noalloc.restype = I
+        L.kron_gptq_quantize_rc_workspace_size.argtypes = [I64, I64, I]
+        L.kron_gptq_quantize_rc_workspace_size.restype = SZ
+        L.kron_gptq_quantize_rc.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, P, SZ, P]
+        L.kron_gptq_quantize_rc.restype = I
+        L.kron_gptq_waterkron_scales.argtypes = [P, I64, P, I64, I, ctypes.c_double, P, P, P]
+        L.kron_gptq_waterkron_scales.restype = I
+        L.kron_gptq_code_entropy_workspace_size.argtypes = [I64]
+        L.kron_gptq_code_entropy_workspace_size.restype = SZ
+        L.kron_gptq_code_entropy.argtypes = [P, I64, P, P, SZ, P]
+        L.kron_gptq_code_entropy.restype = I
         L.kron_gptq_profile_enable.argtypes = [I]
         L.kron_gptq_profile_enable.restype = None
         L.kron_gptq_profile_read.argtypes = [P, P, I, I]
@@ -251,3 +261,76 @@ def kron_gptq_row_scales(W, qmax: int, *, stream=None):
     _raise(L.kron_gptq_row_scales(_ptr(W), m, n, _dtype_code(W), int(qmax), _ptr(s), _stream(stream)),
            "kron_gptq_row_scales")
     return s
+
+
+class RcQuantizer:
+    """Reusable workspace and outputs for repeated solves of one shape on the row- and
+    column-scaled alphabet with unclipped int32 codes (kron_gptq_quantize_rc)."""
+
+    def __init__(self, m: int, n: int, dtype: torch.dtype, device, *, want_E: bool = False):
+        self.m, self.n, self.dtype = int(m), int(n), dtype
+        self.code = KG_F64 if dtype == torch.float64 else KG_F32
+        L = load_library()
+        self.ws = _workspace(L.kron_gptq_quantize_rc_workspace_size(self.m, self.n, self.code), device)
+        self.Z = torch.empty(self.m, self.n, dtype=torch.int32, device=device)
+        self.V = torch.empty(self.m, self.n, dtype=dtype, device=device)
+        self.E = torch.empty(self.m, self.n, dtype=dtype, device=device) if want_E else None
+
+    def run(self, W, U_A, U_B, alpha, beta, stream=None) -> None:
+        """Enqueue one solve on `stream`; does not synchronize."""
+        L = load_library()
+        for t in (W, U_A, U_B, alpha, beta):
+            if t.dtype != self.dtype:
+                raise TypeError("W, U_A, U_B, alpha and beta must all have the solve dtype")
+        _check_dev(W, U_A, U_B, alpha, beta)
+        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or U_B.shape != (self.m, self.m) \
+                or alpha.shape != (self.n,) or beta.shape != (self.m,):
+            raise ValueError("shape mismatch")
+        rc = L.kron_gptq_quantize_rc(_ptr(W), self.m, self.n, self.code, _ptr(U_A), _ptr(U_B), _ptr(alpha),
+                                     _ptr(beta), _ptr(self.Z), _ptr(self.V), _ptr(self.E), _ptr(self.ws),
+                                     self.ws.numel(), _stream(stream))
+        _raise(rc, "kron_gptq_quantize_rc")
+
+    def status(self, stream=None) -> int:
+        return kron_gptq_sync_status(self.ws, stream)
+
+
+def kron_gptq_quantize_rc(W, U_A, U_B, alpha, beta, *, want_E: bool = False, stream=None, check: bool = True):
+    """Two-sided GPTQ of W on the alphabet V = beta alpha^T (.) Z, Z unclipped.
+    Returns (Z int32, V, E or None)."""
+    q = RcQuantizer(W.shape[0], W.shape[1], W.dtype, W.device, want_E=want_E)
+    q.run(W, U_A, U_B, alpha, beta, stream=stream)
+    if check:
+        _raise(q.status(stream), "kron_gptq_quantize_rc (device)")
+    return q.Z, q.V, q.E
+
+
+def kron_gptq_waterkron_scales(U_A, U_B, gamma: float, *, stream=None):
+    """WaterKron steps: alpha = sqrt(gamma) diag(U_A), beta = sqrt(gamma) diag(U_B)."""
+    L = load_library()
+    _check_dev(U_A, U_B)
+    if U_A.dtype != U_B.dtype:
+        raise TypeError("U_A and U_B must share a dtype")
+    n, m = U_A.shape[0], U_B.shape[0]
+    alpha = torch.empty(n, dtype=U_A.dtype, device=U_A.device)
+    beta = torch.empty(m, dtype=U_B.dtype, device=U_B.device)
+    _raise(L.kron_gptq_waterkron_scales(_ptr(U_A), n, _ptr(U_B), m, _dtype_code(U_A), float(gamma), _ptr(alpha),
+                                        _ptr(beta), _stream(stream)), "kron_gptq_waterkron_scales")
+    return alpha, beta
+
+
+ENTROPY_MAX_BINS = (1 << 23) + 1   # every code of the fp32 unclipped alphabet (|Z| < 2^22)
+
+
+def kron_gptq_code_entropy(Z, *, max_bins: int = ENTROPY_MAX_BINS, stream=None) -> float:
+    """Empirical entropy of the int32 codes Z in bits per entry."""
+    L = load_library()
+    _check_dev(Z)
+    if Z.dtype != torch.int32:
+        raise TypeError("Z must be int32")
+    out = torch.empty(1, dtype=torch.float64, device=Z.device)
+    ws = _workspace(L.kron_gptq_code_entropy_workspace_size(int(max_bins)), Z.device)
+    _raise(L.kron_gptq_code_entropy(_ptr(Z), Z.numel(), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "kron_gptq_code_entropy")
+    _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_code_entropy (device)")
+    return float(out.item())

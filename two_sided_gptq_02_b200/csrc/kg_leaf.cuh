@@ -50,8 +50,16 @@ struct LeafSmem {
     Real Rs[KG_T][KG_T + 1];   // R tile as loaded, then the transpose buffer for the final X
                                // (stride 65: column and row walks are both conflict-free)
     Real s[KG_T], invs[KG_T], inva[KG_T], ajj[KG_T];
-    int8_t Cs[KG_T][KG_T];
+    int32_t Cs[KG_T][KG_T];   // codes (int32: the unclipped alphabet needs more than 8 bits)
 };
+
+// Codes leave as int8 (clipped grids) or int32 (the unclipped alphabet), by the caller's width.
+__device__ __forceinline__ void store_code(void* codes, int code_bytes, int64_t idx, int32_t c) {
+    if (code_bytes == 1)
+        static_cast<int8_t*>(codes)[idx] = (int8_t)c;
+    else
+        static_cast<int32_t*>(codes)[idx] = c;
+}
 
 // Store one 16-byte vector; when a second plane is given (fp32 feeding the 3xTF32 update),
 // store the tf32 split instead: hi to dst_hi, the tf32 remainder to dst_lo.
@@ -118,7 +126,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
        Real* __restrict__ XTg, Real* __restrict__ XTlo,
        const Real* __restrict__ UA, int64_t ldA, const Real* __restrict__ UB, int64_t ldB,
        const Real* __restrict__ sp, int qmin, int qmax,
-       int8_t* __restrict__ codes, Real* __restrict__ V, Real* __restrict__ outE) {
+       void* __restrict__ codes, int code_bytes, Real* __restrict__ V, Real* __restrict__ outE) {
     constexpr int T = KG_T;
     constexpr int VW = LeafCfg<Real>::VW;
     constexpr int NC = T / (4 * VW);     // chunks per lane and dot product
@@ -313,7 +321,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
             sm.Es[i][j] = e;
             sm.XT[j][i] = Xv;
             sm.Ws[i][j] = Q;
-            sm.Cs[i][j] = (int8_t)code;
+            sm.Cs[i][j] = (int32_t)code;
         }
         __syncthreads();
     }
@@ -331,7 +339,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
 #pragma unroll
                 for (int u = 0; u < VW; ++u) {
                     if (gj + u < n) {
-                        codes[gi * n + gj + u] = sm.Cs[r][c + u];
+                        store_code(codes, code_bytes, gi * n + gj + u, sm.Cs[r][c + u]);
                         V[gi * n + gj + u] = sm.Ws[r][c + u];
                         if (outE) outE[gi * n + gj + u] = es[u];
                     }

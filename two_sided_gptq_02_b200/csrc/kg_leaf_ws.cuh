@@ -24,7 +24,10 @@
 //     coefficient (b and a are masked to k <= i-4 and k <= j-4), so they cannot change a sum.
 // Hand-off goes through mbarriers, one per ring slot: arrival releases the writer's shared-memory
 // stores, a waiting warp sleeps in try_wait, every wait is bounded in time, and on expiry the CTA
-// records a time-out and skips the rest.  No slot is reused before its previous phase was seen by
+// records a time-out and skips the rest.  Each warp leaves as a whole: a helper warp takes lane
+// 0's verdict; a rounding lane whose wait gives up raises the abort flag and skips its later
+// waits, but still runs every step, so the warp's shuffles stay converged, and the warp votes
+// once, after the last step.  No slot is reused before its previous phase was seen by
 // every waiter: the rounding warp cannot finish step d+8 before both helper groups finished step
 // d+5, and a helper cannot start step d+8 before step d+4 is published.
 #pragma once
@@ -48,12 +51,12 @@ struct LeafWsSmem {
     float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
     float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
     float Ws[KG_T][S];             // w'
-    float Rs[KG_T][KG_T + 1];      // R tile as loaded, then the transpose buffer for the final X
-                                   // (stride 65: column and row walks are both conflict-free)
+    float Rs[KG_T][KG_T + 1];      // R tile as loaded, added to the local X at the end
+                                   // (stride 65: the column walk is conflict-free)
     float colc[KG_T][8];           // column j: a[j-1][j], a[j-2][j], a[j-3][j], 1/a[j][j], a[j][j]
     float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
     float s[KG_T], invs[KG_T];
-    int8_t Cs[KG_T][KG_T];
+    int32_t Cs[KG_T][KG_T];        // codes (int32: the unclipped alphabet needs more than 8 bits)
     uint64_t cbar[WS_RING];        // step d published (32 arrivals)
     uint64_t hbar[WS_RING];        // (P, r') of step d written (one arrival per row)
     int abort_flag;
@@ -97,7 +100,15 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             ws_ldcol(&sm.colc[(unsigned)j < (unsigned)T ? j : 0][0], col[r]);
         }
     };
-    if (!tc::mbar_wait(&sm.hbar[0], 0u, WS_MAX_WAIT_CYCLES, &sm.abort_flag)) return false;
+    bool ok = true;   // this lane's waits so far
+    auto wait_hbar = [&](int d) {
+        if (ok && !tc::mbar_wait(&sm.hbar[d % WS_RING], (uint32_t)((d / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
+                                 &sm.abort_flag)) {
+            ok = false;
+            sm.abort_flag = 1;   // wakes the helpers and the other lanes out of their waits
+        }
+    };
+    wait_hbar(0);
     load_step(0, cpre, ccol);
     float e1[2] = {0.f, 0.f}, e2[2] = {0.f, 0.f}, e3[2] = {0.f, 0.f};   // own E, 1..3 steps ago
     float uo1_1 = 0.f, uo1_2 = 0.f;               // shfl_up(X_odd, 1): X of row 2l-1, 1 and 2 steps ago
@@ -107,9 +118,7 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
     for (int d = 0; d < 2 * T - 1; ++d) {
         // prefetch the next step's inputs; the helpers are normally ahead
         if (d + 1 < 2 * T - 1) {
-            if (!tc::mbar_wait(&sm.hbar[(d + 1) % WS_RING], (uint32_t)(((d + 1) / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
-                               &sm.abort_flag))
-                return false;
+            wait_hbar(d + 1);
             load_step(d + 1, npre, ncol);
         }
         float e[2], X[2], code[2];
@@ -144,7 +153,7 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             if ((unsigned)j < (unsigned)T) {
                 sm.Es[i][j] = e[r];
                 sm.XT[j][i] = X[r];
-                sm.Cs[i][j] = (int8_t)code[r];
+                sm.Cs[i][j] = (int32_t)code[r];
             }
         }
         tc::mbar_arrive(&sm.cbar[d % WS_RING]);
@@ -166,14 +175,14 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             ccol[1][u] = ncol[1][u];
         }
     }
-    return true;
+    return __all_sync(0xffffffffu, ok);
 }
 
 __global__ void __launch_bounds__(WS_THREADS, 1)
 k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, float* __restrict__ Wt,
           float* __restrict__ R, float* __restrict__ Ebuf, float* __restrict__ Elo, float* __restrict__ XTg,
           float* __restrict__ XTlo, const float* __restrict__ UA, int64_t ldA, const float* __restrict__ UB,
-          int64_t ldB, const float* __restrict__ sp, int qmin, int qmax, int8_t* __restrict__ codes,
+          int64_t ldB, const float* __restrict__ sp, int qmin, int qmax, void* __restrict__ codes, int code_bytes,
           float* __restrict__ V, float* __restrict__ outE, DevStatus* status) {
     constexpr int T = KG_T;
     constexpr int VW = 4;
@@ -385,7 +394,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 #pragma unroll
                 for (int u = 0; u < VW; ++u) {
                     if (gj + u < n) {
-                        codes[gi * n + gj + u] = sm.Cs[rr][cc + u];
+                        store_code(codes, code_bytes, gi * n + gj + u, sm.Cs[rr][cc + u]);
                         V[gi * n + gj + u] = (float)sm.Cs[rr][cc + u] * sm.s[rr];
                         if (outE) outE[gi * n + gj + u] = es[u];
                     }
@@ -393,30 +402,19 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             }
         }
     }
-    // ---- the complete X = R + local X: into XTg (X transposed, leading dimension Mp, split for
-    //      the tensor-core update) and back into R (row-major), through the stride-65 buffer
-    //      (independent of the write-back above: no barrier between them)
+    // ---- the complete X = R + local X into XTg (X transposed, leading dimension Mp, split for the
+    //      tensor-core update; independent of the write-back above: no barrier between them).  The
+    //      updates read a solved tile's X only from there, so R itself is not written back.
     for (int idx = tid; idx < T * T; idx += WS_THREADS) {
         const int cc = idx >> 6, rr = idx & 63;
         sm.XT[cc][rr] += sm.Rs[rr][cc];
     }
     __syncthreads();
-    if (helper) {
-        if (XTg) {
-            for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
-                const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
-                leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
-            }
+    if (helper && XTg) {
+        for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
+            const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
+            leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
         }
-        for (int idx = tid; idx < T * T; idx += WS_HELPERS) {
-            const int cc = idx >> 6, rr = idx & 63;
-            sm.Rs[rr][cc] = sm.XT[cc][rr];
-        }
-    }
-    __syncthreads();
-    for (int idx = tid; idx < T * T; idx += WS_THREADS) {
-        const int rr = idx >> 6, cc = idx & 63;
-        R[(r0 + rr) * Np + c0 + cc] = sm.Rs[rr][cc];
     }
 }
 

@@ -156,6 +156,7 @@ extern "C" const char* kron_gptq_status_string(int status) {
         case KG_ERR_NOT_PD: return "factor is not positive definite";
         case KG_ERR_NONFINITE: return "non-finite or non-positive input";
         case KG_ERR_TIMEOUT: return "device wait timed out";
+        case KG_ERR_RANGE: return "code out of the representable range";
         default: return "unknown status";
     }
 }

@@ -25,6 +25,7 @@
 //               W~[I,J] -= sum_{I': I'+J in [D0,mid)} U_B[I',I]^T X[I',J]     (column chain)
 //             Both are dense GEMMs over contiguous K ranges.
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -35,6 +36,7 @@
 #include "kg_leaf_ws.cuh"
 #include "kg_profile.cuh"
 #include "kg_push_tc.cuh"
+#include "kg_rc.cuh"
 
 namespace kg {
 
@@ -43,8 +45,9 @@ constexpr int T = KG_T;
 // ---------------------------------------------------------------------------------------
 // Workspace layout (all offsets 256-byte aligned):
 //   [status 256B][Wt Mp*Np][R Mp*Np][E Mp*Np][scale Mp][UApad Np*Np][UBpad Mp*Mp]
-// Wt holds W minus the column chain, R holds the row chain and, once a tile is solved, its
-// complete X.  The padded factors exist only when m or n is not a multiple of 64; the pad
+// Wt holds W minus the column chain, R holds the row chain of unsolved tiles.  The update reads
+// a solved tile's complete X from R in fp64 and from the split X^T planes (below) in fp32, so
+// only the fp64 leaf writes it back into R.  The padded factors exist only when m or n is not a multiple of 64; the pad
 // is the identity, so padded entries have zero error and never touch real ones.
 // ---------------------------------------------------------------------------------------
 struct QLayout {
@@ -198,7 +201,8 @@ struct QArgs {
     const Real *UA, *UB;
     int64_t ldA, ldB;
     int qmin, qmax;
-    int8_t* codes;
+    void* codes;
+    int code_bytes;   // 1: int8 codes, 4: int32 codes
     Real* V;
     Real* outE;
     cudaStream_t st;
@@ -236,11 +240,11 @@ static int launch_leaf(const QArgs<Real>& a, int D, cudaStream_t st) {
     if constexpr (sizeof(Real) == 4) {
         return launch_k(k_leaf_ws, dim3(ntiles), dim3(WS_THREADS), sizeof(LeafWsSmem), st, true, D, Mt, Nt, a.L.m,
                         a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp,
-                        a.qmin, a.qmax, a.codes, a.V, a.outE, a.status);
+                        a.qmin, a.qmax, a.codes, a.code_bytes, a.V, a.outE, a.status);
     } else {
         return launch_k(k_leaf<Real>, dim3(ntiles), dim3(256), sizeof(LeafSmem<Real>), st, true, D, Mt, Nt, a.L.m,
                         a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB, a.ldB, a.sp,
-                        a.qmin, a.qmax, a.codes, a.V, a.outE);
+                        a.qmin, a.qmax, a.codes, a.code_bytes, a.V, a.outE);
     }
 }
 
@@ -379,9 +383,12 @@ static int solve_all(const QArgs<Real>& a, int ndiag) {
     return rc;
 }
 
+// codes: int8 (code_bytes 1) or int32 (code_bytes 4).  reset_status: clear the status word first;
+// a caller that ran checks of its own into it before the solve passes false.
 template <typename Real>
 static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, const void* UB_, kg_grid grid,
-                         int8_t* codes, void* V, void* outE, void* ws, size_t ws_bytes, cudaStream_t st) {
+                         void* codes, int code_bytes, void* V, void* outE, void* ws, size_t ws_bytes,
+                         cudaStream_t st, bool reset_status = true) {
     const QLayout L = q_layout(m, n, sizeof(Real));
     if (ws_bytes < L.total) return KG_ERR_WORKSPACE;
     unsigned char* base = static_cast<unsigned char*>(ws);
@@ -394,12 +401,13 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
     a.sp = reinterpret_cast<Real*>(base + L.off_s);
     a.qmin = grid.qmin; a.qmax = grid.qmax;
     a.codes = codes;
+    a.code_bytes = code_bytes;
     a.V = static_cast<Real*>(V);
     a.outE = static_cast<Real*>(outE);
     a.st = st;
     a.status = status;
 
-    KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
+    if (reset_status) KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
     const int nb = 148 * 4;
     {
         ProfScope ps(PK_INIT, st);
@@ -541,11 +549,11 @@ extern "C" int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype
     if (dtype == KG_F64) {
         int rc = configure_leaf<double>();
         if (rc) return rc;
-        return quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
+        return quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, 1, out_V, out_E, ws, ws_bytes, st);
     }
     int rc = configure_leaf<float>();
     if (rc) return rc;
-    return quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
+    return quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, 1, out_V, out_E, ws, ws_bytes, st);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -609,14 +617,145 @@ extern "C" int kron_gptq_quantize_noalloc(const void* W, int64_t m, int64_t n, i
         KG_CUDA_TRY(cudaMemsetAsync(scratch, 0, kStatusBytes, st));
     } else if (dtype == KG_F64) {
         rc = configure_leaf<double>();
-        if (!rc) rc = quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, scratch,
+        if (!rc) rc = quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, 1, out_V, out_E, scratch,
                                             (size_t)KG_NOALLOC_SCRATCH_BYTES, st);
     } else {
         rc = configure_leaf<float>();
-        if (!rc) rc = quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, out_V, out_E, scratch,
+        if (!rc) rc = quantize_impl<float>(W, m, n, U_A, U_B, grid, out_codes, 1, out_V, out_E, scratch,
                                            (size_t)KG_NOALLOC_SCRATCH_BYTES, st);
     }
     if (rc) return rc;
     if (dev_status) KG_CUDA_TRY(cudaMemcpyAsync(dev_status, scratch, sizeof(int), cudaMemcpyDeviceToDevice, st));
+    return KG_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Row- and column-scaled alphabet with unclipped integers (kg_rc.cuh): the same solve on the
+// rescaled problem.  Workspace: [the solve's workspace (status word first)][W' m*n][U'_A n*n]
+// [U'_B m*m][unit row scales m], each part 256-byte aligned.
+// ---------------------------------------------------------------------------------------
+namespace kg {
+
+struct RcLayout {
+    size_t off_w, off_ua, off_ub, off_one, total;
+};
+
+static RcLayout rc_layout(int64_t m, int64_t n, size_t es) {
+    RcLayout R{};
+    size_t off = q_layout(m, n, es).total;
+    R.off_w = off;   off = align_up(off + (size_t)(m * n) * es, 256);
+    R.off_ua = off;  off = align_up(off + (size_t)(n * n) * es, 256);
+    R.off_ub = off;  off = align_up(off + (size_t)(m * m) * es, 256);
+    R.off_one = off; off = align_up(off + (size_t)m * es, 256);
+    R.total = off;
+    return R;
+}
+
+// largest |code| the unclipped alphabet represents: fp32 keeps every integer of the step up to
+// 2^24; the margin leaves the rounding of x / s exact in the last bits that matter
+template <typename Real>
+constexpr int32_t rc_bound() { return sizeof(Real) == 4 ? (1 << 22) : (1 << 30); }
+
+template <typename Real>
+static int quantize_rc_impl(const void* W, int64_t m, int64_t n, const void* UA, const void* UB, const void* alpha,
+                            const void* beta, int32_t* Z, void* V, void* E, void* ws, cudaStream_t st) {
+    const RcLayout R = rc_layout(m, n, sizeof(Real));
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    DevStatus* status = reinterpret_cast<DevStatus*>(base);
+    Real* Wp = reinterpret_cast<Real*>(base + R.off_w);
+    Real* UAp = reinterpret_cast<Real*>(base + R.off_ua);
+    Real* UBp = reinterpret_cast<Real*>(base + R.off_ub);
+    Real* one = reinterpret_cast<Real*>(base + R.off_one);
+    const Real* al = static_cast<const Real*>(alpha);
+    const Real* be = static_cast<const Real*>(beta);
+    const int nb = 148 * 4;
+    KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_check_scales<Real><<<nb, 256, 0, st>>>(al, n, be, m, status);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_scale_w<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(W), m, n, al, be, Wp);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_scale_u<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(UA), n, al, UAp);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_scale_u<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(UB), m, be, UBp);
+    }
+    KG_LAUNCH_CHECK();
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_fill<Real><<<std::max<int64_t>(1, std::min<int64_t>(nb, ceil_div(m, 256))), 256, 0, st>>>(one, m, Real(1));
+    }
+    KG_LAUNCH_CHECK();
+    const kg_grid grid{-rc_bound<Real>(), rc_bound<Real>(), one};
+    int rc = quantize_impl<Real>(Wp, m, n, UAp, UBp, grid, Z, 4, V, E, ws, q_layout(m, n, sizeof(Real)).total, st,
+                                 false);
+    if (rc) return rc;
+    {
+        ProfScope ps(PK_INIT, st);
+        k_rc_finish<Real><<<nb, 256, 0, st>>>(Z, m, n, al, be, static_cast<Real*>(V), static_cast<Real*>(E),
+                                              rc_bound<Real>(), status);
+    }
+    KG_LAUNCH_CHECK();
+    return KG_OK;
+}
+
+}  // namespace kg
+
+extern "C" size_t kron_gptq_quantize_rc_workspace_size(int64_t m, int64_t n, int dtype) {
+    if (m < 0 || n < 0) return 0;
+    if (dtype != KG_F32 && dtype != KG_F64) return 0;
+    if (m == 0 || n == 0) return kStatusBytes;
+    return rc_layout(m, n, dtype == KG_F64 ? 8 : 4).total;
+}
+
+extern "C" int kron_gptq_quantize_rc(const void* W, int64_t m, int64_t n, int dtype, const void* U_A,
+                                     const void* U_B, const void* alpha, const void* beta, int32_t* out_Z,
+                                     void* out_V, void* out_E, void* ws, size_t ws_bytes, void* stream) {
+    if (dtype != KG_F32 && dtype != KG_F64) return KG_ERR_UNSUPPORTED;
+    if (m < 0 || n < 0) return KG_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return KG_ERR_ARG;
+    if (m > (int64_t)1 << 20 || n > (int64_t)1 << 20) return KG_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m == 0 || n == 0) {
+        if (ws_bytes < kStatusBytes) return KG_ERR_WORKSPACE;
+        KG_CUDA_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+        return KG_OK;
+    }
+    if (!W || !U_A || !U_B || !alpha || !beta || !out_Z || !out_V) return KG_ERR_ARG;
+    if (ws_bytes < rc_layout(m, n, dtype == KG_F64 ? 8 : 4).total) return KG_ERR_WORKSPACE;
+    if (dtype == KG_F64) {
+        int rc = configure_leaf<double>();
+        if (rc) return rc;
+        return quantize_rc_impl<double>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, st);
+    }
+    int rc = configure_leaf<float>();
+    if (rc) return rc;
+    return quantize_rc_impl<float>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, st);
+}
+
+extern "C" int kron_gptq_waterkron_scales(const void* U_A, int64_t n, const void* U_B, int64_t m, int dtype,
+                                          double gamma, void* alpha, void* beta, void* stream) {
+    if (dtype != KG_F32 && dtype != KG_F64) return KG_ERR_UNSUPPORTED;
+    if (m < 0 || n < 0 || !(gamma > 0.0) || !std::isfinite(gamma)) return KG_ERR_ARG;
+    if (m + n == 0) return KG_OK;
+    if ((n > 0 && (!U_A || !alpha)) || (m > 0 && (!U_B || !beta))) return KG_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int nb = (int)std::max<int64_t>(1, std::min<int64_t>(148 * 4, ceil_div(m + n, 256)));
+    if (dtype == KG_F64)
+        k_wk_scales<double><<<nb, 256, 0, st>>>(static_cast<const double*>(U_A), n, static_cast<const double*>(U_B),
+                                                m, gamma, static_cast<double*>(alpha), static_cast<double*>(beta));
+    else
+        k_wk_scales<float><<<nb, 256, 0, st>>>(static_cast<const float*>(U_A), n, static_cast<const float*>(U_B), m,
+                                               gamma, static_cast<float*>(alpha), static_cast<float*>(beta));
+    KG_LAUNCH_CHECK();
     return KG_OK;
 }
