@@ -50,6 +50,9 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-block", action="store_true")
     ap.add_argument("--no-waterkron", action="store_true")
+    ap.add_argument("--no-onesided", action="store_true")
+    ap.add_argument("--no-factors", action="store_true")
+    ap.add_argument("--no-antidiagonal", action="store_true")
     ap.add_argument("--gamma", type=float, default=0.02, help="WaterKron step knob for the scaled-alphabet line")
     return ap.parse_args()
 
@@ -221,6 +224,98 @@ def _waterkron(kg, torch, spec, Wd, UAd, UBd, gamma, steps, solve_ms, roofline_m
             "mean_E2_over_gamma2_12": mse / (gamma ** 2 / 12.0), "steps": steps,
             "note": "kron_gptq_quantize_rc with kron_gptq_waterkron_scales on the same layer and dtype; "
                     "inputs resident; the step rescaling and the V, E rescaling are inside the time"}
+
+
+def _onesided(kg, torch, spec, Wd, UAd, sd, steps, solve_ms):
+    """One-sided GPTQ (B = I, recursively batched updates) of the same layer, dtype and grid:
+    device time per solve with inputs resident, and the two-sided / one-sided time ratio."""
+    stream = torch.cuda.current_stream()
+    q = kg.OnesidedQuantizer(spec.m, spec.n, Wd.dtype, Wd.device)
+    for _ in range(2):
+        q.run(Wd, UAd, sd, spec.qmin, spec.qmax)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        q.run(Wd, UAd, sd, spec.qmin, spec.qmax)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = q.status()
+    if st != 0:
+        raise kg.KGError(st, "one-sided solve")
+    ms = e0.elapsed_time(e1) / steps
+    # one pass with events around every launch: the leaves against the GEMM updates
+    kg.kron_gptq_profile_read(reset=True)
+    kg.kron_gptq_profile_enable(True)
+    q.run(Wd, UAd, sd, spec.qmin, spec.qmax)
+    torch.cuda.synchronize()
+    kg.kron_gptq_profile_enable(False)
+    prof = kg.kron_gptq_profile_read(reset=True)
+    m, n = spec.m, spec.n
+    return {"ms_per_solve": ms, "weights_per_s": m * n / (ms / 1e3), "two_sided_over_one_sided": solve_ms / ms,
+            "leaf_ms": prof["leaf"][1], "leaf_launches": prof["leaf"][0], "gemm_ms": prof["push"][1],
+            "gemm_launches": prof["push"][0],
+            "gemm_flops": float(m) * n * n, "steps": steps,
+            "note": "kron_gptq_quantize_onesided (64-column leaves + cuBLAS GEMM updates: BF16x9 in fp32, "
+                    "DGEMM in fp64) on the same W, U_A, scales and grid; inputs resident"}
+
+
+def _factors(kg, torch, spec, fp64_peak, reps=3, iters=2, N=4096):
+    """FlipFlop Kronecker factors (iters alternating updates) of the layer's size from N seeded
+    synthetic samples a (N x n), b (N x m), on the device in fp64.  Counted work: the DGEMMs
+    (per side and iteration one N k^2 GEMM for the weights and one for the weighted Gram)."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(int(spec.seed) + 17)
+    a = torch.randn(N, spec.n, generator=gen, device="cuda", dtype=torch.float64)
+    b = torch.randn(N, spec.m, generator=gen, device="cuda", dtype=torch.float64)
+    b *= 1.0 + 0.5 * a[:, :1].abs()
+    kg.kron_gptq_factors(a, b, "flipflop", iters)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kg.kron_gptq_factors(a, b, "flipflop", iters, check=False)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    gemm_flops = iters * 2 * (2.0 * N * spec.n ** 2 + 2.0 * N * spec.m ** 2)
+    return {"method": "flipflop", "iters": iters, "samples": N, "n": spec.n, "m": spec.m, "ms": ms,
+            "gemm_tflops": gemm_flops / (ms / 1e3) / 1e12, "fp64_peak_tflops": fp64_peak,
+            "gemm_frac": gemm_flops / (ms / 1e3) / 1e12 / fp64_peak,
+            "note": "kron_gptq_factors; includes the Cholesky-based inverse factors (kron_gptq_prepare) of every "
+                    "iterate, which gemm_tflops does not count; seeded synthetic samples; median of reps"}
+
+
+def _antidiagonal(kg, torch, spec, W, UA, UB, reps=3):
+    """The non-recursive anti-diagonal baseline (fp64, quartic) against the recursive fp64 solve on
+    the same layer: device time of each (the baseline once, the recursive solve median of reps)."""
+    stream = torch.cuda.current_stream()
+    W64 = W.double().contiguous()
+    s = kg.kron_gptq_row_scales(W64, spec.qmax)
+    q = kg.Quantizer(spec.m, spec.n, torch.float64, W.device)
+    q.run(W64, UA, UB, s, spec.qmin, spec.qmax)
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    fk = statistics.median(timed(lambda: q.run(W64, UA, UB, s, spec.qmin, spec.qmax)) for _ in range(reps))
+    kg.kron_gptq_quantize_antidiagonal(W64, UA, UB, spec.qmin, spec.qmax, s, check=True)   # warm-up
+    anti = timed(lambda: kg.kron_gptq_quantize_antidiagonal(W64, UA, UB, spec.qmin, spec.qmax, s, check=False))
+    m, n = spec.m, spec.n
+    steps = (m + 63) // 64 + (n + 63) // 64 - 1
+    return {"dtype": "f64", "fastkron_ms": fk, "antidiagonal_ms": anti, "antidiagonal_over_fastkron": anti / fk,
+            "antidiagonal_dense_flops": float(steps - 1) * 2.0 * m * n * (m + n),
+            "note": "kron_gptq_quantize_antidiagonal (leaf per tile anti-diagonal + two dense DGEMMs over the "
+                    "whole matrix) vs kron_gptq_quantize, fp64, same layer; inputs resident"}
 
 
 def _traffic(kernel: str, units_per_launch: float):
@@ -490,6 +585,17 @@ def run_ours(args, rank, world, local_rank):
     breakdown = {"push_ms_per_solve": pms / nprof, "leaf_ms_per_solve": lms / nprof, "init_ms_per_solve": ims / nprof,
                  "push_launches_per_solve": pl // nprof, "leaf_launches_per_solve": ll // nprof,
                  "note": "separate pass with CUDA events around every launch"}
+    # latency floor: one dependent entry step t_step (a leaf's time over its 2*64-1 steps, set-up
+    # included), the entry-level chain (m + n - 1) t_step, and the tile-level chain the schedule
+    # runs (every leaf is on the critical path)
+    leaf_launch_ms = (lms / nprof) / max(1, ll // nprof)
+    t_step_us = leaf_launch_ms * 1e3 / (2 * TILE - 1)
+    latency = {"t_step_us": t_step_us, "entry_chain_ms": (m + n - 1) * t_step_us / 1e3,
+               "tile_chain_ms": (ll // nprof) * leaf_launch_ms, "ms_per_step": ms_per_step,
+               "critical_updates_ms": max(0.0, ms_per_step - (ll // nprof) * leaf_launch_ms),
+               "note": "entry_chain_ms: (m+n-1) dependent steps at the leaf's measured step time, the floor of "
+                       "a schedule that overlaps consecutive tile anti-diagonals; tile_chain_ms: the leaves "
+                       "alone; the rest of ms_per_step is the critical-stream update work"}
 
     # ---- end to end: host buffers through the same public call
     e2e = None
@@ -567,6 +673,18 @@ def run_ours(args, rank, world, local_rank):
         waterkron = _waterkron(kg, torch, spec, Wd, UAd, UBd, args.gamma, max(3, min(args.steps, 10)), ms_per_step,
                                solve["roofline_ms"])
 
+    onesided = None
+    if rank == 0 and world == 1 and not args.no_onesided:
+        onesided = _onesided(kg, torch, spec, Wd, UAd, sd, max(3, min(args.steps, 10)), ms_per_step)
+
+    fac = None
+    if rank == 0 and world == 1 and not args.no_factors:
+        fac = _factors(kg, torch, spec, fp64_peak)
+
+    anti = None
+    if rank == 0 and world == 1 and not args.no_antidiagonal:
+        anti = _antidiagonal(kg, torch, spec, W, UA, UB)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(spec, W, A, B, args.damp)
@@ -582,8 +700,10 @@ def run_ours(args, rank, world, local_rank):
                            "l2": "inputs larger than L2 (W, U_A, U_B and a 3-buffer workspace: "
                                  f"{(bytes_compulsory + 3 * m * n * es) / 1e6:.0f} MB)"},
                 "roofline": rl, "roofline_other": rl_other, "solve_roofline": solve, "kernel_breakdown": breakdown,
+                "latency_floor": latency,
                 "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
-                "block": block, "waterkron": waterkron,
+                "block": block, "waterkron": waterkron, "onesided": onesided, "factors": fac,
+                "antidiagonal": anti,
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
                           "source": peak_src}}
         print(json.dumps(line), flush=True)

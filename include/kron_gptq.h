@@ -249,6 +249,76 @@ KG_API int kron_gptq_code_entropy(const int32_t* Z, int64_t count, double* out_b
                                   void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * kron_gptq_quantize_onesided -- standard (one-sided) GPTQ with recursively batched updates
+ *   ("FastKron", Section 2.2: GPTQ, the case B = I of the two-sided algorithm; Section 2.4:
+ *   GPTQ-recursive, solve the first half of the columns, propagate its errors to the second half
+ *   in one batched update, solve the second half).  For column j in order, all rows at once:
+ *       c = clamp(rint(x / s_i), qmin, qmax),  Q = s_i c,  E_ij = (x - Q) / U_A[j,j],
+ *       W[i, j'] -= E_ij U_A[j, j']   for j' > j.
+ *   The result equals kron_gptq_quantize with U_B = I (up to rounding ties).  The recursion stops
+ *   at 64-column blocks; each batched update is a dense GEMM done by cuBLAS on the tensor cores
+ *   (fp32: BF16x9 emulation of fp32; fp64: DGEMM), with its workspace inside ws.  cuBLAS keeps one
+ *   handle per host thread and device, created on the first call (cublasCreate allocates its own
+ *   small device state then; nothing else is allocated).
+ * Arguments: W (m x n), U_A (n x n, 16-byte aligned), grid, out_codes (int8), out_V, out_E
+ *   (optional): as kron_gptq_quantize.  ws: kron_gptq_quantize_onesided_workspace_size(m, n, dtype) bytes,
+ *   256-byte aligned, status word first.
+ * m == 0 or n == 0 is a no-op returning KG_OK.
+ * Device errors: KG_ERR_NONFINITE (NaN/Inf in W, a scale or a diagonal entry of U_A not > 0).
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_quantize_onesided_workspace_size(int64_t m, int64_t n, int dtype);
+KG_API int kron_gptq_quantize_onesided(const void* W, int64_t m, int64_t n, int dtype,
+                                       const void* U_A, kg_grid grid,
+                                       int8_t* out_codes, void* out_V, void* out_E,
+                                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_factors -- Kronecker factors A (n x n), B (m x m) with A (x) B ~ H = E[a a^T (x) b b^T]
+ *   from N samples: a_k the input of the linear unit (length n), b_k the gradient at its output
+ *   (length m) ("FastKron", Section 3.2 and Appendix E.2; "WaterKron and FlipFlop Hessian",
+ *   Table 1 and Section 5).  E is the sample mean.
+ *     KG_FACTOR_MARGINAL:  A = E[a a^T], B = E[b b^T].
+ *     KG_FACTOR_FROBENIUS: from B = I, repeat: A = E[(b^T B b) a a^T] / ||B||_F^2,
+ *                          B = E[(a^T A a) b b^T] / ||A||_F^2  (least squares on ||H - A (x) B||_F).
+ *     KG_FACTOR_FLIPFLOP:  from B = I, repeat: A = E[(b^T B^-1 b) a a^T] / m,
+ *                          B = E[(a^T A^-1 a) b b^T] / n.
+ *   iters (>= 1) is the number of (A, B) updates of the two alternating methods.  Computed in
+ *   fp64: DGEMMs (cuBLAS, workspace inside ws) and the library's own prepare for A^-1, B^-1.
+ * Arguments:
+ *   a, b      device, row-major N x n and N x m, dtype KG_F32 (promoted) or KG_F64.
+ *   A, B      device fp64 outputs, n x n and m x m, symmetric.
+ *   ws        kron_gptq_factors_workspace_size(N, n, m) bytes, 256-byte aligned, status first.
+ * Device errors: KG_ERR_NONFINITE (NaN/Inf in a or b), KG_ERR_NOT_PD (FlipFlop: an iterate that is
+ *   not positive definite, e.g. fewer samples than n or m).
+ * --------------------------------------------------------------------------------------- */
+typedef enum kg_factor_method {
+    KG_FACTOR_MARGINAL = 0,
+    KG_FACTOR_FROBENIUS = 1,
+    KG_FACTOR_FLIPFLOP = 2
+} kg_factor_method;
+KG_API size_t kron_gptq_factors_workspace_size(int64_t N, int64_t n, int64_t m);
+KG_API int kron_gptq_factors(const void* a, const void* b, int64_t N, int64_t n, int64_t m, int dtype,
+                             int method, int iters, double* A, double* B,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_quantize_antidiagonal -- the non-recursive anti-diagonal algorithm ("FastKron",
+ *   Section 2.3, FastKron-antidiagonal; the scheme YAQA uses): the tile anti-diagonals are solved in
+ *   order, and after each one its errors reach the whole matrix through the dense product
+ *   W -= U_B^T Delta U_A (Delta = the errors of that anti-diagonal).  Same outputs as
+ *   kron_gptq_quantize (equal codes up to rounding ties: the FastKron variants are equivalent,
+ *   Section 2.5), at O(mn(m+n)) work per anti-diagonal -- quartic in total.  A baseline to measure
+ *   the recursion against; fp64 only, dense products in cuBLAS (DGEMM) with a workspace slice.
+ * Arguments: as kron_gptq_quantize with dtype KG_F64; m, n <= 2^17.
+ *   ws: kron_gptq_quantize_antidiagonal_workspace_size(m, n) bytes, 256-byte aligned.
+ * --------------------------------------------------------------------------------------- */
+KG_API size_t kron_gptq_quantize_antidiagonal_workspace_size(int64_t m, int64_t n);
+KG_API int kron_gptq_quantize_antidiagonal(const void* W, int64_t m, int64_t n,
+                                           const void* U_A, const void* U_B, kg_grid grid,
+                                           int8_t* out_codes, void* out_V, void* out_E,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Diagnostics (tracing).  The library counts every kernel launch by kind:
  *   0 init/validation, 1 in-tile sweep (leaf), 2 trailing band update (push),
  *   3 factor preparation, 4 loss and scales, 5 persistent whole-solve kernel.

@@ -15,6 +15,9 @@ Public functions mirror the C names:
                                               alphabet, unclipped codes)
     kron_gptq_waterkron_scales(U_A, U_B, gamma)     -> alpha, beta (WaterKron steps)
     kron_gptq_code_entropy(Z)                       -> bits per entry
+    kron_gptq_quantize_onesided(W, U_A, ...)        -> codes (int8), V, E  (one-sided GPTQ, B = I)
+    kron_gptq_factors(a, b, method, iters)          -> A, B (Kronecker factors from samples)
+    kron_gptq_quantize_antidiagonal(W, U_A, U_B, ...) -> codes, V, E (quartic baseline, fp64)
     kron_gptq_sync_status(ws, stream)      -> device status word
 """
 from __future__ import annotations
@@ -25,6 +28,7 @@ from ._lib import (  # noqa: F401
     KGError,
     Quantizer,
     RcQuantizer,
+    OnesidedQuantizer,
     PROFILE_KINDS,
     kron_gptq_loss,
     kron_gptq_profile_enable,
@@ -33,6 +37,9 @@ from ._lib import (  # noqa: F401
     kron_gptq_quantize,
     kron_gptq_quantize_noalloc,
     kron_gptq_quantize_rc,
+    kron_gptq_quantize_onesided,
+    kron_gptq_factors,
+    kron_gptq_quantize_antidiagonal,
     kron_gptq_code_entropy,
     kron_gptq_waterkron_scales,
     kron_gptq_row_scales,

@@ -77,6 +77,18 @@ def load_library():
         L.kron_gptq_code_entropy_workspace_size.restype = SZ
         L.kron_gptq_code_entropy.argtypes = [P, I64, P, P, SZ, P]
         L.kron_gptq_code_entropy.restype = I
+        L.kron_gptq_quantize_onesided_workspace_size.argtypes = [I64, I64, I]
+        L.kron_gptq_quantize_onesided_workspace_size.restype = SZ
+        L.kron_gptq_quantize_onesided.argtypes = [P, I64, I64, I, P, _Grid, P, P, P, P, SZ, P]
+        L.kron_gptq_quantize_onesided.restype = I
+        L.kron_gptq_factors_workspace_size.argtypes = [I64, I64, I64]
+        L.kron_gptq_factors_workspace_size.restype = SZ
+        L.kron_gptq_factors.argtypes = [P, P, I64, I64, I64, I, I, I, P, P, P, SZ, P]
+        L.kron_gptq_factors.restype = I
+        L.kron_gptq_quantize_antidiagonal_workspace_size.argtypes = [I64, I64]
+        L.kron_gptq_quantize_antidiagonal_workspace_size.restype = SZ
+        L.kron_gptq_quantize_antidiagonal.argtypes = [P, I64, I64, P, P, _Grid, P, P, P, P, SZ, P]
+        L.kron_gptq_quantize_antidiagonal.restype = I
         L.kron_gptq_profile_enable.argtypes = [I]
         L.kron_gptq_profile_enable.restype = None
         L.kron_gptq_profile_read.argtypes = [P, P, I, I]
@@ -334,3 +346,91 @@ def kron_gptq_code_entropy(Z, *, max_bins: int = ENTROPY_MAX_BINS, stream=None) 
            "kron_gptq_code_entropy")
     _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_code_entropy (device)")
     return float(out.item())
+
+
+class OnesidedQuantizer:
+    """Reusable workspace and outputs for repeated one-sided GPTQ solves of one shape
+    (kron_gptq_quantize_onesided)."""
+
+    def __init__(self, m: int, n: int, dtype: torch.dtype, device, *, want_E: bool = False):
+        self.m, self.n, self.dtype = int(m), int(n), dtype
+        self.code = KG_F64 if dtype == torch.float64 else KG_F32
+        L = load_library()
+        self.ws = _workspace(L.kron_gptq_quantize_onesided_workspace_size(self.m, self.n, self.code), device)
+        self.codes = torch.empty(self.m, self.n, dtype=torch.int8, device=device)
+        self.V = torch.empty(self.m, self.n, dtype=dtype, device=device)
+        self.E = torch.empty(self.m, self.n, dtype=dtype, device=device) if want_E else None
+
+    def run(self, W, U_A, row_scale, qmin: int, qmax: int, stream=None) -> None:
+        L = load_library()
+        for t in (W, U_A, row_scale):
+            if t.dtype != self.dtype:
+                raise TypeError("W, U_A and row_scale must all have the solve dtype")
+        _check_dev(W, U_A, row_scale)
+        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or row_scale.shape != (self.m,):
+            raise ValueError("shape mismatch")
+        grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
+        rc = L.kron_gptq_quantize_onesided(_ptr(W), self.m, self.n, self.code, _ptr(U_A), grid, _ptr(self.codes),
+                                           _ptr(self.V), _ptr(self.E), _ptr(self.ws), self.ws.numel(),
+                                           _stream(stream))
+        _raise(rc, "kron_gptq_quantize_onesided")
+
+    def status(self, stream=None) -> int:
+        return kron_gptq_sync_status(self.ws, stream)
+
+
+def kron_gptq_quantize_onesided(W, U_A, qmin: int, qmax: int, row_scale, *, want_E: bool = False, stream=None,
+                                check: bool = True):
+    """One-sided GPTQ of W (the case B = I).  Returns (codes int8, V, E or None)."""
+    q = OnesidedQuantizer(W.shape[0], W.shape[1], W.dtype, W.device, want_E=want_E)
+    q.run(W, U_A, row_scale, qmin, qmax, stream=stream)
+    if check:
+        _raise(q.status(stream), "kron_gptq_quantize_onesided (device)")
+    return q.codes, q.V, q.E
+
+
+FACTOR_METHODS = {"marginal": 0, "frobenius": 1, "flipflop": 2}
+
+
+def kron_gptq_factors(a, b, method: str = "flipflop", iters: int = 2, *, stream=None, check: bool = True):
+    """Kronecker factors (A n x n, B m x m, fp64) of E[a a^T (x) b b^T] from samples a (N x n) and
+    b (N x m): "marginal", "frobenius" or "flipflop" (iters alternating updates from B = I)."""
+    L = load_library()
+    _check_dev(a, b)
+    if a.dtype != b.dtype:
+        raise TypeError("a and b must share a dtype")
+    N, n = a.shape
+    if b.shape[0] != N:
+        raise ValueError("a and b need the same number of samples")
+    m = b.shape[1]
+    A = torch.empty(n, n, dtype=torch.float64, device=a.device)
+    B = torch.empty(m, m, dtype=torch.float64, device=a.device)
+    ws = _workspace(L.kron_gptq_factors_workspace_size(N, n, m), a.device)
+    rc = L.kron_gptq_factors(_ptr(a), _ptr(b), N, n, m, _dtype_code(a), FACTOR_METHODS[method], int(iters), _ptr(A),
+                             _ptr(B), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "kron_gptq_factors")
+    if check:
+        _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_factors (device)")
+    return A, B
+
+
+def kron_gptq_quantize_antidiagonal(W, U_A, U_B, qmin: int, qmax: int, row_scale, *, want_E: bool = False,
+                                    stream=None, check: bool = True):
+    """The non-recursive anti-diagonal baseline (quartic work; fp64).  Same outputs as
+    kron_gptq_quantize: (codes int8, V, E or None)."""
+    L = load_library()
+    _check_dev(W, U_A, U_B, row_scale)
+    if W.dtype != torch.float64:
+        raise TypeError("the anti-diagonal baseline runs in fp64")
+    m, n = W.shape
+    ws = _workspace(L.kron_gptq_quantize_antidiagonal_workspace_size(m, n), W.device)
+    codes = torch.empty(m, n, dtype=torch.int8, device=W.device)
+    V = torch.empty(m, n, dtype=W.dtype, device=W.device)
+    E = torch.empty(m, n, dtype=W.dtype, device=W.device) if want_E else None
+    grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
+    rc = L.kron_gptq_quantize_antidiagonal(_ptr(W), m, n, _ptr(U_A), _ptr(U_B), grid, _ptr(codes), _ptr(V), _ptr(E),
+                                           _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "kron_gptq_quantize_antidiagonal")
+    if check:
+        _raise(L.kron_gptq_sync_status(_ptr(ws), _stream(stream)), "kron_gptq_quantize_antidiagonal (device)")
+    return codes, V, E

@@ -21,6 +21,7 @@ LIB = os.path.join(HERE, "libkrongptq.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+CUDA_LIB = os.path.join(os.path.dirname(os.path.dirname(NVCC)), "lib64")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
           "-Xcompiler", "-fvisibility=hidden"]
@@ -48,7 +49,10 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
             changed = True
     if changed:
         tmp = LIB + f".{os.getpid()}.tmp"
-        subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
+        # cuBLAS (the one-sided path's plain GEMM) is linked dynamically; a process that imported
+        # torch first already holds a libcublas.so.12 and the loader reuses it
+        subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lcublas",
+                               "-Xlinker", "-rpath", "-Xlinker", CUDA_LIB])
         os.replace(tmp, LIB)
     return LIB
 

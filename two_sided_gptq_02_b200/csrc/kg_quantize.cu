@@ -30,6 +30,7 @@
 #include <utility>
 #include <vector>
 
+#include "kg_blas.cuh"
 #include "kg_common.cuh"
 #include "kg_gemm.cuh"
 #include "kg_leaf.cuh"
@@ -383,12 +384,16 @@ static int solve_all(const QArgs<Real>& a, int ndiag) {
     return rc;
 }
 
+template <typename Real>
+static int solve_antidiagonal(const QArgs<Real>& a, int ndiag, unsigned char* extra);
+
 // codes: int8 (code_bytes 1) or int32 (code_bytes 4).  reset_status: clear the status word first;
-// a caller that ran checks of its own into it before the solve passes false.
+// a caller that ran checks of its own into it before the solve passes false.  anti_extra: when
+// given, the solve is the non-recursive anti-diagonal baseline (fp64) with its extra workspace.
 template <typename Real>
 static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, const void* UB_, kg_grid grid,
                          void* codes, int code_bytes, void* V, void* outE, void* ws, size_t ws_bytes,
-                         cudaStream_t st, bool reset_status = true) {
+                         cudaStream_t st, bool reset_status = true, unsigned char* anti_extra = nullptr) {
     const QLayout L = q_layout(m, n, sizeof(Real));
     if (ws_bytes < L.total) return KG_ERR_WORKSPACE;
     unsigned char* base = static_cast<unsigned char*>(ws);
@@ -475,6 +480,7 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         }
         KG_LAUNCH_CHECK();
     }
+    if (anti_extra) return solve_antidiagonal(a, (int)(L.Mt + L.Nt - 1), anti_extra);
     return solve_all(a, (int)(L.Mt + L.Nt - 1));
 }
 
@@ -758,4 +764,98 @@ extern "C" int kron_gptq_waterkron_scales(const void* U_A, int64_t n, const void
                                                gamma, static_cast<float*>(alpha), static_cast<float*>(beta));
     KG_LAUNCH_CHECK();
     return KG_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// The non-recursive anti-diagonal algorithm ("FastKron", Section 2.3, FastKron-antidiagonal; the
+// scheme of YAQA): after each tile anti-diagonal D is solved, its errors reach the whole matrix at
+// once through the dense product  W~ -= U_B^T Delta_D U_A,  Delta_D = E on the tiles of D and zero
+// elsewhere.  Every step costs two full GEMMs, O(mn(m+n)), so the total is quartic; it exists as
+// the baseline the recursion is measured against.  fp64 only.  The leaves are the solver's own:
+// the row-chain buffer R stays zero (every cross-tile contribution is already in W~), so a leaf
+// propagates only its own tile's errors, which the dense product then applies a second time to
+// entries the leaf has finished -- entries nobody reads again.
+// ---------------------------------------------------------------------------------------
+namespace kg {
+
+constexpr size_t ANTI_BLAS_WS = 32u << 20;
+
+static size_t anti_extra_bytes(int64_t m, int64_t n) {
+    const QLayout L = q_layout(m, n, 8);
+    return 2 * align_up((size_t)(L.Mp * L.Np) * 8, 256) + ANTI_BLAS_WS;
+}
+
+// Delta = E on the tiles of anti-diagonal D, zero elsewhere (Mp x Np, row-major like E)
+__global__ void k_anti_delta(const double* __restrict__ E, int D, int64_t Mp, int64_t Np, double* __restrict__ Dl) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < Mp * Np; p += stride) {
+        const int64_t i = p / Np, j = p - i * Np;
+        Dl[p] = (i / KG_T + j / KG_T == D) ? E[p] : 0.0;
+    }
+}
+
+template <typename Real>
+static int solve_antidiagonal(const QArgs<Real>& a, int ndiag, unsigned char* extra) {
+    if constexpr (sizeof(Real) != 8) {
+        return KG_ERR_UNSUPPORTED;
+    } else {
+        const int64_t Mp = a.L.Mp, Np = a.L.Np;
+        double* Dl = reinterpret_cast<double*>(extra);
+        double* T = reinterpret_cast<double*>(extra + align_up((size_t)(Mp * Np) * 8, 256));
+        void* bws = extra + 2 * align_up((size_t)(Mp * Np) * 8, 256);
+        cublasHandle_t h;
+        int rc = blas_handle(&h);
+        if (!rc) rc = blas_bind(h, a.st, bws, ANTI_BLAS_WS);
+        if (rc) return rc;
+        const double one = 1.0, zero = 0.0, minus_one = -1.0;
+        const int nb = 148 * 4;
+        for (int D = 0; D < ndiag; ++D) {
+            if ((rc = launch_leaf(a, D, a.st))) return rc;
+            if (D + 1 == ndiag) break;
+            {
+                ProfScope ps(PK_PUSH, a.st);
+                k_anti_delta<<<nb, 256, 0, a.st>>>(a.E, D, Mp, Np, Dl);
+                KG_LAUNCH_CHECK();
+                // T = Delta U_A:  column-major T^T = U_A^T Delta^T (row-major storage read as its transpose)
+                if (cublasDgemm(h, CUBLAS_OP_N, CUBLAS_OP_N, (int)Np, (int)Mp, (int)Np, &one, a.UA, (int)a.ldA, Dl,
+                                (int)Np, &zero, T, (int)Np) != CUBLAS_STATUS_SUCCESS)
+                    return KG_ERR_CUDA;
+                // W~ -= U_B^T T:  column-major W~^T -= T^T U_B
+                if (cublasDgemm(h, CUBLAS_OP_N, CUBLAS_OP_T, (int)Np, (int)Mp, (int)Mp, &minus_one, T, (int)Np, a.UB,
+                                (int)a.ldB, &one, a.Wt, (int)Np) != CUBLAS_STATUS_SUCCESS)
+                    return KG_ERR_CUDA;
+            }
+        }
+        return KG_OK;
+    }
+}
+
+}  // namespace kg
+
+extern "C" size_t kron_gptq_quantize_antidiagonal_workspace_size(int64_t m, int64_t n) {
+    if (m < 0 || n < 0) return 0;
+    if (m == 0 || n == 0) return kStatusBytes;
+    return q_layout(m, n, 8).total + anti_extra_bytes(m, n);
+}
+
+extern "C" int kron_gptq_quantize_antidiagonal(const void* W, int64_t m, int64_t n, const void* U_A, const void* U_B,
+                                               kg_grid grid, int8_t* out_codes, void* out_V, void* out_E, void* ws,
+                                               size_t ws_bytes, void* stream) {
+    if (m < 0 || n < 0) return KG_ERR_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return KG_ERR_ARG;
+    if (grid.qmin >= 0 || grid.qmax <= 0 || grid.qmin < -128 || grid.qmax > 127) return KG_ERR_UNSUPPORTED;
+    if (m > (int64_t)1 << 17 || n > (int64_t)1 << 17) return KG_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m == 0 || n == 0) {
+        if (ws_bytes < kStatusBytes) return KG_ERR_WORKSPACE;
+        KG_CUDA_TRY(cudaMemsetAsync(ws, 0, kStatusBytes, st));
+        return KG_OK;
+    }
+    if (!W || !U_A || !U_B || !grid.row_scale || !out_codes || !out_V) return KG_ERR_ARG;
+    const size_t qbytes = q_layout(m, n, 8).total;
+    if (ws_bytes < qbytes + anti_extra_bytes(m, n)) return KG_ERR_WORKSPACE;
+    int rc = configure_leaf<double>();
+    if (rc) return rc;
+    return quantize_impl<double>(W, m, n, U_A, U_B, grid, out_codes, 1, out_V, out_E, ws, qbytes, st, true,
+                                 static_cast<unsigned char*>(ws) + qbytes);
 }
