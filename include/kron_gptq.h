@@ -18,7 +18,10 @@
  * Conventions for every call:
  *   - All matrices are dense, row-major, contiguous, in DEVICE memory owned by the caller.
  *     The library never allocates or frees device memory: each call takes a caller-owned
- *     workspace of at least the size the matching *_workspace_size() function returns.
+ *     workspace of at least the size the matching *_workspace_size() function returns.  The one
+ *     exception: the calls that hand a plain dense GEMM to cuBLAS (quantize_onesided, factors,
+ *     quantize_antidiagonal) create one cuBLAS handle per host thread and device on first use,
+ *     and cuBLAS allocates its own small device state then; their GEMM workspace is inside ws.
  *   - Calls are asynchronous on the given CUDA stream (passed as void*, a cudaStream_t;
  *     NULL = the legacy default stream).  Errors the host can see (bad arguments,
  *     unsupported options, a failed launch) are returned at once and nothing is launched
