@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.kron_gptq_version() >= 10000
-    for code in range(0, -8, -1):
+    for code in range(0, -9, -1):
         s = lib.kron_gptq_status_string(code).decode()
         assert s and s != "unknown status"
     assert lib.kron_gptq_status_string(-99).decode() == "unknown status"
@@ -90,6 +90,50 @@ def test_host_side_argument_errors(lib):
     assert lib.kron_gptq_loss(fake, fake, 4, 4, 1, fake, fake, 1, 0.0, fake, fake, 8, None) == -4
     assert lib.kron_gptq_row_scales(fake, 4, 4, 1, 0, fake, None) == -1
     assert lib.kron_gptq_sync_status(None, None) == -1
+
+
+def test_host_side_argument_errors_of_the_next_rows(lib):
+    from two_sided_gptq_02_b200._lib import _Grid
+    P = ctypes.c_void_p
+    fake = P(256 * 1000)
+    big = 1 << 40
+    g = _Grid(-4, 3, fake)
+    # scaled alphabet: dtype, sizes, workspace alignment, null steps, small workspace
+    rc = lib.kron_gptq_quantize_rc
+    assert rc(fake, 8, 8, 5, fake, fake, fake, fake, fake, fake, None, fake, big, None) == -2
+    assert rc(fake, -1, 8, 1, fake, fake, fake, fake, fake, fake, None, fake, big, None) == -1
+    assert rc(fake, 8, 8, 1, fake, fake, fake, fake, fake, fake, None, P(300), big, None) == -1
+    assert rc(fake, 8, 8, 1, fake, fake, None, fake, fake, fake, None, fake, big, None) == -1
+    assert rc(fake, 64, 64, 1, fake, fake, fake, fake, fake, fake, None, fake, 4096, None) == -4
+    assert lib.kron_gptq_quantize_rc_workspace_size(64, 64, 1) > lib.kron_gptq_quantize_workspace_size(64, 64, 1)
+    assert lib.kron_gptq_waterkron_scales(fake, 8, fake, 8, 1, -1.0, fake, fake, None) == -1
+    assert lib.kron_gptq_waterkron_scales(fake, 8, fake, 8, 1, float("nan"), fake, fake, None) == -1
+    assert lib.kron_gptq_waterkron_scales(fake, 8, fake, 8, 3, 0.1, fake, fake, None) == -2
+    # entropy: count, output, workspace, the 32-bit counters
+    ent = lib.kron_gptq_code_entropy
+    assert ent(fake, -1, fake, fake, big, None) == -1
+    assert ent(fake, 10, None, fake, big, None) == -1
+    assert ent(fake, 10, fake, P(7), big, None) == -1
+    assert ent(fake, 10, fake, fake, 16, None) == -4
+    assert ent(fake, 1 << 32, fake, fake, big, None) == -2
+    assert lib.kron_gptq_code_entropy_workspace_size(1000) >= 256 + 4000
+    # one-sided: grid, misaligned U_A, small workspace
+    os_ = lib.kron_gptq_quantize_onesided
+    assert os_(fake, 8, 8, 1, fake, _Grid(-4, 300, fake), fake, fake, None, fake, big, None) == -2
+    assert os_(fake, 8, 8, 1, P(256 * 1000 + 4), g, fake, fake, None, fake, big, None) == -1
+    assert os_(fake, 64, 64, 1, fake, g, fake, fake, None, fake, 4096, None) == -4
+    # factors: method, sizes, iterations, workspace
+    fac = lib.kron_gptq_factors
+    assert fac(fake, fake, 10, 4, 4, 2, 7, 1, fake, fake, fake, big, None) == -2
+    assert fac(fake, fake, 0, 4, 4, 2, 2, 1, fake, fake, fake, big, None) == -1
+    assert fac(fake, fake, 10, 4, 4, 2, 2, 0, fake, fake, fake, big, None) == -1
+    assert fac(fake, fake, 10, 4, 4, 2, 2, 1, fake, fake, fake, 1024, None) == -4
+    assert lib.kron_gptq_factors_workspace_size(0, 4, 4) == 0
+    # anti-diagonal baseline: grid, sizes, workspace
+    an = lib.kron_gptq_quantize_antidiagonal
+    assert an(fake, 8, 8, fake, fake, _Grid(1, 3, fake), fake, fake, None, fake, big, None) == -2
+    assert an(fake, 1 << 18, 8, fake, fake, g, fake, fake, None, fake, big, None) == -2
+    assert an(fake, 64, 64, fake, fake, g, fake, fake, None, fake, 4096, None) == -4
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
