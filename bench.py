@@ -318,6 +318,33 @@ def _antidiagonal(kg, torch, spec, W, UA, UB, reps=3):
                     "whole matrix) vs kron_gptq_quantize, fp64, same layer; inputs resident"}
 
 
+def _host():
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def _cpu_cubic(spec, W, UA, UB):
+    """The cubic CPU baseline (oracle.quantize_cubic: the two-chain form entry by entry, OpenMP over
+    each anti-diagonal's entries, all host cores) on the full layer, fp64."""
+    import oracle
+    Wn = W.double().cpu().numpy()
+    UAn, UBn = UA.double().cpu().numpy(), UB.double().cpu().numpy()
+    s = oracle.row_scales(Wn, spec.qmax)
+    t0 = time.perf_counter()
+    oracle.quantize_cubic(Wn, UAn, UBn, s, spec.qmin, spec.qmax)
+    t = time.perf_counter() - t0
+    return {"value": spec.m * spec.n / t, "unit": "weights/s", "seconds": t, "cores": oracle.cubic_threads(),
+            "kind": "cubic two-chain CPU baseline (oracle.quantize_cubic)", "sample": f"the full {spec.m}x{spec.n} layer"}
+
+
 def _traffic(kernel: str, units_per_launch: float):
     """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/traffic.json):
     bytes per unit of work (a tile for the leaves) x the units one launch processes on average.
@@ -464,7 +491,8 @@ def run_reference(args, rank, world):
             "config": {"workload": args.workload, "m": spec.m, "n": spec.n, "bits": spec.bits,
                        "sample": vals[0]["sample"]},
             "cpu_baseline": {"value": v, "unit": "weights/s", "cores": 1, "kind": "oracle", "sample": vals[0]["sample"]},
-            "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "host": _host()}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -686,8 +714,10 @@ def run_ours(args, rank, world, local_rank):
         anti = _antidiagonal(kg, torch, spec, W, UA, UB)
 
     cpu = None
+    cubic = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(spec, W, A, B, args.damp)
+        cubic = _cpu_cubic(spec, W, UA, UB)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
@@ -703,7 +733,7 @@ def run_ours(args, rank, world, local_rank):
                 "latency_floor": latency,
                 "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
                 "block": block, "waterkron": waterkron, "onesided": onesided, "factors": fac,
-                "antidiagonal": anti,
+                "antidiagonal": anti, "cpu_cubic": cubic, "host": _host(),
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_derived": tf32_peak,
                           "source": peak_src}}
         print(json.dumps(line), flush=True)

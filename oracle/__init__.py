@@ -21,6 +21,8 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
                   one-sided GPTQ of W^T, transpose symmetry, leading-block invariance,
                   loss identity, error bound, certificate.
   quantize_onesided  pinned: the vectorized form with B=I, RTN when A is diagonal.
+  quantize_cubic  pinned: equals quantize_naive (codes exactly away from ties, E to 1e-9) on
+                  ragged shapes; a plain reorganisation of the same sums (the CPU baseline).
   loss            pinned: closed forms (sum E^2) and numpy einsum of the definition.
   quantize_rc     pinned: literal vectorized form with a per-entry step (4x4, 6x5, ...),
                   A=B=I reduces to per-entry rounding, alpha=1 / beta=s equals
@@ -55,7 +57,7 @@ def build(force: bool = False) -> str:
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".{os.getpid()}.tmp"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fopenmp",
                                "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
@@ -77,6 +79,10 @@ def _load():
             lib.ora_quantize_naive.restype = I64
             lib.ora_quantize_rc.argtypes = [P, I64, I64, P, P, P, P, P, ctypes.c_double, P, P, P, P, P]
             lib.ora_quantize_rc.restype = I64
+            lib.ora_quantize_cubic.argtypes = [P, I64, I64, P, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
+            lib.ora_quantize_cubic.restype = ctypes.c_int
+            lib.ora_threads.argtypes = []
+            lib.ora_threads.restype = ctypes.c_int
             lib.ora_quantize_onesided.argtypes = [P, I64, I64, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
             lib.ora_quantize_onesided.restype = None
             lib.ora_rtn.argtypes = [P, I64, I64, P, ctypes.c_int, ctypes.c_int, P, P]
@@ -140,6 +146,24 @@ def quantize_naive(W, UA, UB, s, qmin: int, qmax: int, *, forced=None, tol: floa
     if nb < 0:
         raise MemoryError("oracle quantize: allocation failed")
     return dict(codes=codes, V=V, E=E, t=t, boundary=bflag.astype(bool), n_boundary=int(nb))
+
+
+def quantize_cubic(W, UA, UB, s, qmin: int, qmax: int):
+    """The cubic CPU baseline: the two-chain form over anti-diagonals, OpenMP over each one's
+    entries (all host cores).  Returns dict(codes, V, E)."""
+    W, UA, UB, s = _f64(W), _f64(UA), _f64(UB), _f64(s)
+    m, n = W.shape
+    codes = np.zeros((m, n), dtype=np.int32)
+    V = np.zeros((m, n), dtype=np.float64)
+    E = np.zeros((m, n), dtype=np.float64)
+    if _load().ora_quantize_cubic(_ptr(W), m, n, _ptr(UA), _ptr(UB), _ptr(s), int(qmin), int(qmax), _ptr(codes),
+                                  _ptr(V), _ptr(E)) != 0:
+        raise MemoryError("oracle quantize_cubic: allocation failed")
+    return dict(codes=codes, V=V, E=E)
+
+
+def cubic_threads() -> int:
+    return int(_load().ora_threads())
 
 
 NOT_FORCED_64 = -(2 ** 63)

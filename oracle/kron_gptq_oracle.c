@@ -311,3 +311,57 @@ double ora_loss(const double* W, const double* V, const double* Ad, const double
     free(D);
     return (double)acc;
 }
+
+/* ------------------------------------------------------------------------------------
+ * The cubic CPU baseline: the same algorithm in its two-chain form, entry by entry over the
+ * anti-diagonals d = i + j, the entries of one anti-diagonal in parallel (OpenMP) -- no tiles,
+ * no batching.  Two-chain reading of the batched update W -= U_B^T E U_A ("FastKron",
+ * Sections 2.3-2.4): the error of entry (i,j) enters later entries of its row through
+ *     R[i][j'] += E_ij U_A[j][j']                       (j' > j, the row chain)
+ * and, once (i,j) is solved, its complete X_ij = R[i][j] + E_ij U_A[j][j] enters later entries of
+ * its column through
+ *     W~[i'][j] -= U_B[i][i'] X_ij                       (i' > i, the column chain),
+ * so that x = W~[i][j] - U_B[i][i] R[i][j].  Work mn(m+n)/2 multiply-adds; the entries of one
+ * anti-diagonal write disjoint rows of R and disjoint columns of W~ (kept transposed, WT[j][i]).
+ * Rounding as in ora_quantize_naive.  Returns 0, or -1 when memory runs out.
+ * ------------------------------------------------------------------------------------ */
+int ora_quantize_cubic(const double* W, int64_t m, int64_t n,
+                       const double* UA, const double* UB, const double* s,
+                       int qmin, int qmax, int32_t* codes, double* V, double* E)
+{
+    double* WT = (double*)malloc(sizeof(double) * (size_t)(m * n));
+    double* R = (double*)calloc((size_t)(m * n), sizeof(double));
+    if (!WT || !R) { free(WT); free(R); return -1; }
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) WT[j * m + i] = W[i * n + j];
+    for (int64_t d = 0; d < m + n - 1; ++d) {
+        const int64_t i0 = d - n + 1 > 0 ? d - n + 1 : 0;
+        const int64_t i1 = d < m - 1 ? d : m - 1;
+#pragma omp parallel for schedule(static)
+        for (int64_t i = i0; i <= i1; ++i) {
+            const int64_t j = d - i;
+            const int64_t p = i * n + j;
+            const double* ra = UA + j * n;             /* row j of U_A */
+            const double* rb = UB + i * m;             /* row i of U_B */
+            double* rr = R + i * n;                    /* row i of R */
+            double* wc = WT + j * m;                   /* column j of W~ */
+            const double x = wc[i] - rb[i] * rr[j];
+            const double c = ora_clamp(rint(x / s[i]), qmin, qmax);
+            const double q = s[i] * c;
+            const double e = (x - q) / (rb[i] * ra[j]);
+            codes[p] = (int32_t)c;
+            V[p] = q;
+            if (E) E[p] = e;
+            const double X = rr[j] + e * ra[j];
+            for (int64_t jp = j + 1; jp < n; ++jp) rr[jp] += e * ra[jp];
+            for (int64_t ip = i + 1; ip < m; ++ip) wc[ip] -= rb[ip] * X;
+        }
+    }
+    free(WT);
+    free(R);
+    return 0;
+}
+
+/* threads the OpenMP loops of ora_quantize_cubic use */
+#include <omp.h>
+int ora_threads(void) { return omp_get_max_threads(); }

@@ -441,3 +441,18 @@ def test_planted_mistakes_fail_an_rc_pin(mutation):
     cert = oracle.certificate_rc(*args, c, V, E)
     caught = (not np.array_equal(c, lit["codes"])) or cert["resid_rel"] > 1e-9 or cert["code_mismatch"] > 0
     assert caught, mutation
+
+
+# ---------------------------------------------------------------- the cubic CPU baseline
+@pytest.mark.parametrize("m,n,seed,bits", [(6, 5, 1, 4), (40, 33, 2, 3), (127, 129, 3, 3), (200, 70, 4, 2), (1, 90, 5, 4)])
+def test_cubic_baseline_equals_the_definition(m, n, seed, bits):
+    # the two-chain, anti-diagonal-parallel form reorganises the same sums: equal codes away from
+    # rounding ties, E to rounding noise
+    f = _factors(m, n, seed, bits=bits)
+    r = oracle.quantize_naive(f["W"], f["UA"], f["UB"], f["s"], f["qmin"], f["qmax"])
+    c = oracle.quantize_cubic(f["W"], f["UA"], f["UB"], f["s"], f["qmin"], f["qmax"])
+    assert r["n_boundary"] == 0
+    np.testing.assert_array_equal(c["codes"], r["codes"])
+    np.testing.assert_array_equal(c["V"], r["V"])
+    np.testing.assert_allclose(c["E"], r["E"], rtol=1e-9, atol=1e-12 * np.abs(r["E"]).max())
+    assert oracle.cubic_threads() >= 1
