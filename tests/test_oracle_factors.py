@@ -108,3 +108,102 @@ def test_first_iterations_share_A_and_differ_in_B():
     Ap, Bp = factors.flipflop(a, b, 1)
     np.testing.assert_allclose(Af, Ap, rtol=1e-13)
     assert not np.allclose(Bf / np.trace(Bf), Bp / np.trace(Bp))
+
+
+# ---- planted mistakes: a mutated copy of each estimator must fail one of the pins above ----
+# (A slip in the constant of the A update alone is not a mistake: the B update that follows is the
+# exact least-squares or flip-flop step for that A, so only the split of scale between the two
+# factors moves, which two-sided GPTQ does not see.)
+
+def _mutated(mutation):
+    """Copies of marginal / frobenius / flipflop / hessian with one plausible slip planted."""
+    def gram(x, w, d):
+        return (x.T * w) @ x / d
+
+    def marginal(a, b):
+        d = a.shape[0] - 1 if mutation == "marginal_unbiased" else a.shape[0]
+        return gram(a, np.ones(a.shape[0]), d), gram(b, np.ones(b.shape[0]), d)
+
+    def frobenius(a, b, iters=1):
+        B = np.eye(b.shape[1])
+        for _ in range(iters):
+            Bw = np.eye(b.shape[1]) if mutation == "frob_drop_B_weight" else B
+            w = np.einsum("ki,ij,kj->k", b, Bw, b)
+            A = gram(a, w, a.shape[0]) / np.sum(B * B)
+            v = np.einsum("ki,ij,kj->k", a, A, a)
+            c = np.sqrt(np.sum(A * A)) if mutation == "frob_norm_not_squared" else np.sum(A * A)
+            B = gram(b, v, b.shape[0]) / c
+        return A, B
+
+    def flipflop(a, b, iters=1):
+        n, m = a.shape[1], b.shape[1]
+        cA, cB = (n, m) if mutation == "flip_swapped_dims" else (m, n)
+        B = np.eye(m)
+        for _ in range(iters):
+            Bi = B if mutation == "flip_no_inverse" else np.linalg.inv(B)
+            A = gram(a, np.einsum("ki,ij,kj->k", b, Bi, b), a.shape[0]) / cA
+            v = np.einsum("ki,ij,kj->k", a, np.linalg.inv(A), a)
+            B = gram(b, v, b.shape[0]) / cB
+        return A, B
+
+    def hessian(a, b):
+        H = 0
+        for k in range(a.shape[0]):
+            pa, pb = np.outer(a[k], a[k]), np.outer(b[k], b[k])
+            H = H + (np.kron(pb, pa) if mutation == "kron_order_swapped" else np.kron(pa, pb))
+        return H / a.shape[0]
+
+    return marginal, frobenius, flipflop, hessian
+
+
+def _pins_hold(marginal, frobenius, flipflop, hessian):
+    """The checks of the pins above, as one predicate over a set of estimators."""
+    a, b = _samples(7, 3, 2, 0)
+    H = hessian(a, b)
+    if not np.isclose(H[1 * 2 + 0, 2 * 2 + 1], np.mean(a[:, 1] * a[:, 2] * b[:, 0] * b[:, 1]), rtol=1e-12):
+        return False
+    rng = np.random.default_rng(1)
+    ai, bj = rng.standard_normal((5, 4)), rng.standard_normal((6, 3))
+    a, b = np.repeat(ai, 6, axis=0), np.tile(bj, (5, 1))
+    H = hessian(a, b)
+    for A, B in (marginal(a, b), frobenius(a, b, 1), flipflop(a, b, 1)):
+        if not np.allclose(np.kron(A, B), H, rtol=1e-9, atol=1e-12):
+            return False
+    a, b = _samples(200, 4, 3, 2)
+    H = hessian(a, b)
+    s = np.linalg.svd(factors.rearrange(H, 4, 3), compute_uv=False)
+    A, B = frobenius(a, b, 60)
+    if not np.isclose(np.sum((H - np.kron(A, B)) ** 2), np.sum(s ** 2) - s[0] ** 2, rtol=1e-8):
+        return False
+    a, b = _samples(300, 4, 3, 3)
+    H = hessian(a, b)
+    A, B = flipflop(a, b, 200)
+    f0 = factors.mismatch(H, A, B)
+    rng = np.random.default_rng(4)
+    Ah, Bh = np.linalg.cholesky(A), np.linalg.cholesky(B)
+    for _ in range(20):
+        Sa = rng.standard_normal((4, 4)); Sa = 0.5 * (Sa + Sa.T)
+        Sb = rng.standard_normal((3, 3)); Sb = 0.5 * (Sb + Sb.T)
+        A2 = Ah @ (np.eye(4) + 1e-2 * Sa) @ Ah.T
+        B2 = Bh @ (np.eye(3) + 1e-2 * Sb) @ Bh.T
+        if factors.mismatch(H, A2, B2) < f0 * (1 - 1e-12):
+            return False
+    return True
+
+
+def test_unmutated_copy_passes_the_pins():
+    assert _pins_hold(*_mutated(None))
+    a, b = _samples(40, 4, 3, 9)
+    m0, f0, p0, h0 = _mutated(None)
+    for mine, ref in ((m0(a, b), factors.marginal(a, b)), (f0(a, b, 3), factors.frobenius(a, b, 3)),
+                      (p0(a, b, 3), factors.flipflop(a, b, 3))):
+        np.testing.assert_allclose(mine[0], ref[0], rtol=1e-12)
+        np.testing.assert_allclose(mine[1], ref[1], rtol=1e-12)
+    np.testing.assert_allclose(h0(a, b), factors.hessian(a, b), rtol=1e-12)
+
+
+@pytest.mark.parametrize("mutation", ["marginal_unbiased", "frob_drop_B_weight", "frob_norm_not_squared",
+                                      "flip_no_inverse", "flip_swapped_dims", "kron_order_swapped"])
+def test_planted_mistakes_fail_a_factor_pin(mutation):
+    with np.errstate(all="ignore"):     # a mutated iteration may run off to inf / nan
+        assert not _pins_hold(*_mutated(mutation)), mutation
