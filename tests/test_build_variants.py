@@ -37,3 +37,23 @@ def test_default_build_does_not_contain_the_paired_leaf(tmp_path):
                          text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-3000:]
     assert "k_leaf_pair" not in out.stdout and "kron_gptq_debug_pair_timeline" not in out.stdout
+
+
+def test_variant_library_builds_apart_and_loads(tmp_path):
+    """build.py --define/--out: a variant library of its own, loadable on the host, exporting the
+    timeline reader, while the default library keeps its own objects."""
+    import ctypes
+    import subprocess
+    import sys
+    out = tmp_path / "libkrongptq_pair.so"
+    r = subprocess.run([sys.executable, "-m", "two_sided_gptq_02_b200.build", "--define", "KG_EXPERIMENTAL_PAIR",
+                        "--define", "KG_PAIR_TIMELINE", "--out", str(out)], cwd=ROOT, capture_output=True,
+                       text=True, timeout=1200)
+    assert r.returncode == 0, r.stderr[-3000:]
+    assert out.exists() and (tmp_path / "libkrongptq_pair_objs" / "flags.txt").read_text().endswith(
+        "-DKG_EXPERIMENTAL_PAIR -DKG_PAIR_TIMELINE")
+    lib = ctypes.CDLL(str(out))
+    assert lib.kron_gptq_version() > 0
+    assert hasattr(lib, "kron_gptq_debug_pair_timeline")
+    default = ctypes.CDLL(os.path.join(ROOT, "two_sided_gptq_02_b200", "libkrongptq.so"))
+    assert not hasattr(default, "kron_gptq_debug_pair_timeline")

@@ -31,7 +31,8 @@ class _Grid(ctypes.Structure):
 
 
 def lib_path() -> str:
-    return os.path.join(_HERE, "libkrongptq.so")
+    """The in-tree library, or the build that KRON_GPTQ_LIB names (a variant built with --out)."""
+    return os.environ.get("KRON_GPTQ_LIB") or os.path.join(_HERE, "libkrongptq.so")
 
 
 def load_library():

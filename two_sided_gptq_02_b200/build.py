@@ -1,14 +1,19 @@
 """Build the kron_gptq CUDA library (libkrongptq.so) in-tree for sm_100a.
 
     python -m two_sided_gptq_02_b200.build [--force] [--verbose]
+    python -m two_sided_gptq_02_b200.build --define KG_EXPERIMENTAL_PAIR --out <path>.so
 
 Each .cu under csrc/ is compiled separately (so an unchanged file is not rebuilt) and the
 objects are linked into a shared library next to this file.  Flags: sm_100a only,
 -O3, -lineinfo; no fast-math (rounding decisions must follow IEEE semantics).
+A variant (--define NAME, repeatable) is built into the library named by --out, with its objects
+in a folder of their own, and leaves the default library alone; the binding loads it when
+KRON_GPTQ_LIB names it.
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -31,13 +36,21 @@ def _deps(src: str) -> list[str]:
     return [src] + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "kron_gptq.h")]
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    lib = os.path.abspath(out) if out else LIB
+    # objects of a variant live beside its library, so that the default objects are never mixed in
+    objdir = BUILD if lib == LIB else os.path.splitext(lib)[0] + "_objs"
+    os.makedirs(objdir, exist_ok=True)
+    # objects built with other flags are stale (the stamp is written once every object is built)
+    stamp, flags = os.path.join(objdir, "flags.txt"), " ".join(CFLAGS + (extra or []))
+    if not os.path.exists(stamp) or open(stamp).read() != flags:
+        force = True
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    objs = []
-    changed = force or not os.path.exists(LIB)
+    objs, jobs = [], []
+    changed = force or not os.path.exists(lib)
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         newest = max(os.path.getmtime(d) for d in _deps(src))
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < newest:
@@ -45,22 +58,33 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
                 print(" ".join(cmd), flush=True)
-            subprocess.check_call(cmd)
-            changed = True
+            jobs.append(cmd)
+    if jobs:
+        # one nvcc per translation unit, in parallel
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as pool:
+            for f in [pool.submit(subprocess.check_call, cmd) for cmd in jobs]:
+                f.result()
+        changed = True
+    with open(stamp, "w") as f:
+        f.write(flags)
     if changed:
-        tmp = LIB + f".{os.getpid()}.tmp"
+        tmp = lib + f".{os.getpid()}.tmp"
         # cuBLAS (the one-sided path's plain GEMM) is linked dynamically; a process that imported
         # torch first already holds a libcublas.so.12 and the loader reuses it
         subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lcublas",
                                "-Xlinker", "-rpath", "-Xlinker", CUDA_LIB])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--define", action="append", default=[], help="preprocessor macro of a variant build")
+    ap.add_argument("--out", default=None, help="library path of a variant build")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    if a.define and not a.out:
+        ap.error("a variant (--define) needs its own --out library path")
+    print(build(force=a.force, verbose=a.verbose, extra=[f"-D{d}" for d in a.define], out=a.out))
     sys.exit(0)
