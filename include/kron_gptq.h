@@ -132,7 +132,8 @@ KG_API int kron_gptq_prepare(const void* A, int64_t n, const void* B, int64_t m,
  *   ws        kron_gptq_quantize_workspace_size(m, n, dtype) bytes, 256-byte aligned.
  * m == 0 or n == 0 is a no-op returning KG_OK.
  * Device errors: KG_ERR_NONFINITE (NaN/Inf in W or scales, non-positive scale or factor
- *   diagonal), KG_ERR_TIMEOUT (a bounded wait in the persistent kernel ran out).
+ *   diagonal), KG_ERR_TIMEOUT (a bounded device-side wait ran out: the hand-off between the
+ *   warps of a leaf, or the load / MMA pipeline of an update).
  * --------------------------------------------------------------------------------------- */
 KG_API size_t kron_gptq_quantize_workspace_size(int64_t m, int64_t n, int dtype);
 KG_API int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype,
@@ -324,7 +325,7 @@ KG_API int kron_gptq_quantize_antidiagonal(const void* W, int64_t m, int64_t n,
 /* ---------------------------------------------------------------------------------------
  * Diagnostics (tracing).  The library counts every kernel launch by kind:
  *   0 init/validation, 1 in-tile sweep (leaf), 2 trailing band update (push),
- *   3 factor preparation, 4 loss and scales, 5 persistent whole-solve kernel.
+ *   3 factor preparation, 4 loss and scales, 5 reserved (no launch of this kind).
  * kron_gptq_profile_enable(1) additionally brackets each launch with a pair of CUDA events
  * recorded on the launch's own stream (the events are host-side resources; no device
  * memory is allocated).  kron_gptq_profile_read() waits for the recorded events, adds

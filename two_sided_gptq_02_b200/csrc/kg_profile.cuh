@@ -16,7 +16,7 @@ enum ProfKind : int {
     PK_PUSH = 2,     // trailing band updates (row and column chains)
     PK_PREPARE = 3,  // factor preparation kernels
     PK_LOSS = 4,     // loss and scale kernels
-    PK_SOLVE = 5,    // persistent whole-solve kernel
+    PK_SOLVE = 5,    // reserved: no launch of this kind
     PK_COUNT = 8
 };
 
