@@ -39,13 +39,18 @@ def _deps(src: str) -> list[str]:
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
           out: str | None = None) -> str:
     lib = os.path.abspath(out) if out else LIB
+    if lib == LIB and any(f.startswith("-D") for f in (extra or [])):
+        raise ValueError("a variant build (-D...) needs its own library path (out=...)")
     # objects of a variant live beside its library, so that the default objects are never mixed in
     objdir = BUILD if lib == LIB else os.path.splitext(lib)[0] + "_objs"
     os.makedirs(objdir, exist_ok=True)
     # objects built with other flags are stale (the stamp is written once every object is built)
     stamp, flags = os.path.join(objdir, "flags.txt"), " ".join(CFLAGS + (extra or []))
-    if not os.path.exists(stamp) or open(stamp).read() != flags:
+    if not os.path.exists(stamp):
         force = True
+    else:
+        with open(stamp) as f:
+            force = force or f.read() != flags
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     objs, jobs = [], []
     changed = force or not os.path.exists(lib)
