@@ -22,6 +22,8 @@
  *     exception: the calls that hand a plain dense GEMM to cuBLAS (quantize_onesided, factors,
  *     quantize_antidiagonal) create one cuBLAS handle per host thread and device on first use,
  *     and cuBLAS allocates its own small device state then; their GEMM workspace is inside ws.
+ *     Handles live until the process exits, also those of threads that have ended, so make
+ *     these calls from long-lived threads.
  *   - Calls are asynchronous on the given CUDA stream (passed as void*, a cudaStream_t;
  *     NULL = the legacy default stream).  Errors the host can see (bad arguments,
  *     unsupported options, a failed launch) are returned at once and nothing is launched

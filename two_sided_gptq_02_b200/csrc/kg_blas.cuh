@@ -1,6 +1,9 @@
 // kg_blas.cuh -- the library's cuBLAS handle: one per host thread and device, created on the
 // first call that needs a plain dense GEMM and kept for the life of the process.  Callers set the
-// stream and hand cuBLAS a workspace slice before every use.
+// stream and hand cuBLAS a workspace slice before every use.  Handles are never destroyed: a
+// destructor at thread or process exit could run after the CUDA runtime has shut down, so the
+// handle of a thread that exits stays allocated.  Callers that spawn many short-lived threads
+// should make these calls from a long-lived one.
 #pragma once
 
 #include <cublas_v2.h>
