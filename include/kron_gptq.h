@@ -30,6 +30,12 @@
  *     after them.  Errors only the device can see (a factor that is not positive definite,
  *     non-finite input, a device wait that ran out) are written to a status word inside the
  *     workspace; kron_gptq_sync_status() synchronizes the stream and returns it.
+ *   - The recursive two-sided solves (quantize, quantize_noalloc, quantize_rc) run part of
+ *     their update work on a second, internal stream; the caller's stream waits for it at the
+ *     end, so each call stays one asynchronous operation on the caller's stream.  For this
+ *     each host thread keeps, per device, eight
+ *     non-blocking streams and their events (host-side driver objects, no device buffers),
+ *     created on the first call and kept until the process exits.
  *   - Concurrent calls on different streams need distinct workspaces.
  *   - Status codes: 0 = success, negative = error (see kg_status).
  */

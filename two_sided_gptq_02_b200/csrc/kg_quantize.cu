@@ -368,9 +368,10 @@ static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
 }
 
 // Per host thread and device: a few bulk streams with their events, created on first use and kept
-// for the life of the process.  Calls take them in turn, so that solves in flight at the same time
-// on different caller streams (several layers at once) also run their bulk updates side by side;
-// two calls that share a slot only serialise their bulk work.
+// for the life of the process (a thread that exits leaves its slots allocated; nothing is destroyed
+// at exit, when the CUDA runtime may already be gone).  Calls take them in turn, so that solves in
+// flight at the same time on different caller streams (several layers at once) also run their bulk
+// updates side by side; two calls that share a slot only serialise their bulk work.
 struct SchedSlot {
     cudaStream_t bulk = nullptr;
     cudaEvent_t fork = nullptr;
