@@ -39,6 +39,18 @@ def test_library_exports_every_declared_symbol(lib):
     assert not missing, missing
 
 
+def test_library_exports_only_declared_entry_points(lib):
+    """No undeclared kron_gptq_* symbol (a debug entry point of a variant build) in the default
+    library."""
+    import shutil
+    import subprocess
+    if not shutil.which("nm"):
+        pytest.skip("nm not found")
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True, check=True)
+    exported = {ln.split()[-1] for ln in out.stdout.splitlines() if ln.split() and ln.split()[-1].startswith("kron_gptq_")}
+    assert exported == set(_declared()), sorted(exported ^ set(_declared()))
+
+
 def test_version_and_status_strings(lib):
     assert lib.kron_gptq_version() >= 10000
     for code in range(0, -9, -1):
