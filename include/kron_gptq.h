@@ -118,8 +118,8 @@ KG_API int kron_gptq_prepare(const void* A, int64_t n, const void* B, int64_t m,
 
 /* ---------------------------------------------------------------------------------------
  * kron_gptq_quantize -- two-sided GPTQ rounding of W ("FastKron" Sec. 2.2-2.5).
- *   Produces the codes of the naive algorithm: entries visited in any order consistent with
- *   "top-left first"; for entry (i,j) with current value x:
+ *   Produces the codes of the naive algorithm: every entry is visited after all entries to
+ *   its top-left (any such order gives the same result); for entry (i,j) with current value x:
  *       c = clamp(rint(x / s_i), qmin, qmax),  Q = s_i c,
  *       E_ij = (x - Q) / (U_B[i,i] U_A[j,j]),
  *       W[i',j'] -= U_B[i,i'] E_ij U_A[j,j']   for i' >= i, j' >= j, (i',j') != (i,j).

@@ -11,7 +11,7 @@ Section 5).  Three approximations H ~ A (x) B, all float64:
     E[(a^T A a) b b^T] / ||A||_F^2.
   * FlipFlop (the same alternation with the reciprocal weighting, the Gaussian flip-flop):
     A = E[(b^T B^-1 b) a a^T] / m,  B = E[(a^T A^-1 a) b b^T] / n.
-Both iterations start from B = I (Table 1: "starting from the identity matrix"); one iteration
+Both iterations start from B = I (Table 1 starts them from the identity); one iteration
 updates A, then B.  The normalisations (a reading: the pages' displayed formulas were lost) fix
 only the split of a common scale between A and B, which two-sided GPTQ does not see.
 

@@ -29,7 +29,7 @@
  *  - U_A is the upper-triangular Cholesky factor of A_d^{-1} (U_A^T U_A = A_d^{-1}),
  *    U_B likewise; kron(U_A, U_B) is then the upper Cholesky factor of kron(A_d,B_d)^{-1}.
  *  - damping: A_d = A + damp * mean(diag A) * I, each factor with its own mean [WK Sec. 2
- *    ("a small damping kappa I can be added")].
+ *    allows adding a small multiple of the identity to each factor].
  *  - quantize(x) = s_i * clamp(rint(x / s_i), qmin, qmax), rint = round half to even.
  */
 #include <math.h>
@@ -40,8 +40,9 @@
 #define ORA_NOT_FORCED INT32_MIN
 
 /* ------------------------------------------------------------------------------------
- * Factor preparation [WK Sec. 2 Notation; FK Sec. 2.6: "computing the inverse and the
- * Cholesky decomposition of the Hessian"].  Four textbook steps, in this order:
+ * Factor preparation [WK Sec. 2 Notation; FK Sec. 2.6: the inverse of each factor and a
+ * Cholesky factorisation of it are a separate step before the rounding].  Four textbook steps,
+ * in this order:
  *   1. A_d = A + damp * mean(diag A) * I
  *   2. L   = Cholesky(A_d)               (lower, L L^T = A_d)
  *   3. A_d^{-1} = L^{-T} L^{-1}          (via the inverse of L by forward substitution)
@@ -113,7 +114,7 @@ done:
 
 /* Per-row scale s_i = max_j |W_ij| / qmax; an all-zero row gets scale 1 so that its
  * codes are 0.  The scales are chosen up front from the original W, before any update
- * [WK Sec. 2.4: "those scaling factors are chosen up front and handed to the algorithm"]. */
+ * [WK Sec. 2.4: the scales are fixed before the rounding starts and passed in]. */
 void ora_row_scales(const double* W, int64_t m, int64_t n, int qmax, double* s)
 {
     for (int64_t i = 0; i < m; ++i) {
@@ -279,8 +280,8 @@ void ora_quantize_onesided(const double* W, int64_t m, int64_t n, const double* 
     free(Wt);
 }
 
-/* Round to nearest on the grid, no error feedback [FK Sec. 1: "simply rounding each
- * entry ... is suboptimal"]; per-entry scale S. */
+/* Round to nearest on the grid, no error feedback [FK Sec. 1: the baseline that GPTQ-style
+ * error feedback improves on]; per-entry scale S. */
 void ora_rtn(const double* W, int64_t m, int64_t n, const double* S, int qmin, int qmax,
              int32_t* codes, double* V)
 {
