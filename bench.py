@@ -53,6 +53,8 @@ def _args():
     ap.add_argument("--no-onesided", action="store_true")
     ap.add_argument("--no-factors", action="store_true")
     ap.add_argument("--no-antidiagonal", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (fp64 4096x4096, fp32 14336x4096 and 4096x14336)")
     ap.add_argument("--gamma", type=float, default=0.02, help="WaterKron step knob for the scaled-alphabet line")
     return ap.parse_args()
 
@@ -316,6 +318,81 @@ def _antidiagonal(kg, torch, spec, W, UA, UB, reps=3):
             "antidiagonal_dense_flops": float(steps - 1) * 2.0 * m * n * (m + n),
             "note": "kron_gptq_quantize_antidiagonal (leaf per tile anti-diagonal + two dense DGEMMs over the "
                     "whole matrix) vs kron_gptq_quantize, fp64, same layer; inputs resident"}
+
+
+def _prepare_flops(n, m):
+    """FLOPs of kron_gptq_prepare per factor pair: a Cholesky (k^3/3) and a triangular inverse
+    (k^3/3) of each k x k factor; the damping, the output copies and the fp32 rounding are O(k^2)."""
+    return 2.0 / 3.0 * (float(n) ** 3 + float(m) ** 3)
+
+
+def _time_prepare(kg, torch, A, B, damp, fp64_peak, reps=3):
+    """kron_gptq_prepare (damping, reversed Cholesky and triangular inverse of A and B, fp64, with
+    the fp32 copies the fp32 solve uses): device time, median of reps (CUDA events on the stream)."""
+    stream = torch.cuda.current_stream()
+    kg.kron_gptq_prepare(A, B, damp)   # warm-up, checked
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kg.kron_gptq_prepare(A, B, damp, check=False)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    fl = _prepare_flops(A.shape[0], B.shape[0])
+    return {"ms": ms, "n": int(A.shape[0]), "m": int(B.shape[0]), "flops": fl, "tflops": fl / (ms / 1e3) / 1e12,
+            "fp64_peak_tflops": fp64_peak, "frac_of_fp64": fl / (ms / 1e3) / 1e12 / fp64_peak,
+            "note": "kron_gptq_prepare(A, B, damp) with fp32 copies, inputs resident; FLOPs 2/3 (n^3 + m^3) "
+                    "(Cholesky and triangular inverse of each factor); fraction of the cuBLAS DGEMM rate "
+                    "measured in this run; median of reps"}
+
+
+def _config_line(kg, torch, name, dtype, damp, steps, fp64_peak, tf32_peak, hbm, cubic):
+    """One more workload of the pages' shapes: the solve (device time with inputs resident, median
+    over steps), its solve-roofline fraction, kron_gptq_prepare of its factors, and (cubic) the
+    cubic CPU baseline on the full layer."""
+    from synth_inputs.layers import layer_inputs, workload
+    spec = workload(name)[0]
+    dt = torch.float32 if dtype == "f32" else torch.float64
+    W, A, B = layer_inputs(spec, device="cuda")
+    prep = _time_prepare(kg, torch, A, B, damp, fp64_peak)
+    UA, UB, UA32, UB32 = kg.kron_gptq_prepare(A, B, damp)
+    del A, B
+    Wd, UAd, UBd = (W.float().contiguous(), UA32, UB32) if dt == torch.float32 else (W, UA, UB)
+    sd = kg.kron_gptq_row_scales(Wd, spec.qmax)
+    q = kg.Quantizer(spec.m, spec.n, dt, Wd.device)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        q.run(Wd, UAd, UBd, sd, spec.qmin, spec.qmax)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q.run(Wd, UAd, UBd, sd, spec.qmin, spec.qmax)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    st = q.status()
+    if st != 0:
+        raise kg.KGError(st, f"{name} solve")
+    ms = statistics.median(times)
+    m, n = spec.m, spec.n
+    es = 4 if dt == torch.float32 else 8
+    p_tensor = tf32_peak / 3.0 if dt == torch.float32 else fp64_peak
+    t_roof = max(2.0 * m * n * (m + n) / (p_tensor * 1e12), (es * (2 * m * n + n * n + m * m + m) + m * n) / (hbm * 1e9))
+    out = {"workload": f"{name}: {m}x{n} (out x in), {spec.bits}-bit", "dtype": dtype, "ms_per_solve": ms,
+           "weights_per_s": m * n / (ms / 1e3), "solve_roofline_ms": t_roof * 1e3,
+           "solve_roofline_frac": t_roof * 1e3 / ms, "p_tensor_tflops": p_tensor, "prepare": prep,
+           "prepare_plus_solve_ms": prep["ms"] + ms, "steps": steps,
+           "note": "inputs resident; CUDA events around each solve, median; roofline as the headline's "
+                   "(TF32/3 for fp32, DGEMM for fp64, measured in this run)"}
+    if cubic:
+        out["cpu_cubic"] = _cpu_cubic(spec, W, UA, UB)
+    del q, Wd, UAd, UBd, W, UA, UB, UA32, UB32
+    torch.cuda.empty_cache()
+    return out
 
 
 def _host():
@@ -601,7 +678,7 @@ def run_ours(args, rank, world, local_rank):
     if dt == torch.float32:
         push_rl = {"bound": "tensor", "achieved": push_achieved, "peak": tf32_peak / 3.0, "unit": "TFLOP/s",
                    "frac": push_achieved / (tf32_peak / 3.0), "traffic": None, "kernel": "k_push_tc32",
-                   "peak_source": f"3xTF32: {peak_src} bf16 burst x 1.1/2.25 (nominal TF32/bf16 ratio) / 3",
+                   "peak_source": "3xTF32: cuBLAS fp32 GEMM with TF32 allowed, 8192^3, measured in this run / 3",
                    "frac_of_raw_tf32": 3.0 * push_achieved / tf32_peak}
         leaf_rl = {"bound": "alu", "achieved": leaf_achieved, "peak": FP32_SIMT_PEAK_TFLOPS, "unit": "TFLOP/s",
                    "frac": leaf_achieved / FP32_SIMT_PEAK_TFLOPS, "traffic": None, "kernel": "k_leaf_ws",
@@ -728,6 +805,21 @@ def run_ours(args, rank, world, local_rank):
         cpu = _cpu_baseline(spec, W, A, B, args.damp)
         cubic = _cpu_cubic(spec, W, UA, UB)
 
+    prep = None
+    configs = None
+    if rank == 0 and world == 1:
+        prep = _time_prepare(kg, torch, A, B, args.damp, fp64_peak)
+        prep["prepare_plus_solve_ms"] = prep["ms"] + ms_per_step
+        if not args.no_configs:
+            del W, A, B, UA, UB
+            torch.cuda.empty_cache()
+            other = [("sq4096", "f64"), ("ffn_up", "f32"), ("ffn_down", "f32")]
+            if args.workload != "sq4096" or args.dtype != "f32":
+                other = [("sq4096", "f32")] + [c for c in other if c != (args.workload, args.dtype)]
+            configs = [_config_line(kg, torch, nm, dt_, args.damp, max(3, min(args.steps, 10)), fp64_peak, tf32_peak,
+                                    hbm, cubic=not args.no_cpu_baseline and nm != "sq4096")
+                       for nm, dt_ in other if (nm, dt_) != (args.workload, args.dtype)]
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -742,7 +834,7 @@ def run_ours(args, rank, world, local_rank):
                 "latency_floor": latency,
                 "clocks": clocks, "gpu_launches": int(gpu_launches), "e2e": e2e, "cpu_baseline": cpu,
                 "block": block, "waterkron": waterkron, "onesided": onesided, "factors": fac,
-                "antidiagonal": anti, "cpu_cubic": cubic, "host": _host(),
+                "antidiagonal": anti, "cpu_cubic": cubic, "prepare": prep, "configs": configs, "host": _host(),
                 "peaks": {"hbm_gbs": hbm, "fp64_tflops_measured": fp64_peak, "tf32_tflops_measured": tf32_peak,
                           "tf32_tflops_derived": tf32_derived,
                           "source": peak_src}}

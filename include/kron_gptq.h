@@ -191,7 +191,10 @@ KG_API int kron_gptq_sync_status(const void* ws, void* stream);
  *     operands for the tensor cores, and 24 in fp64: fp32 fits e.g. 896 x 896, fp64 e.g.
  *     1024 x 1024).
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream capture.
+ *     with that device current).  The first call from each host thread on a device also creates
+ *     the eight internal bulk streams and their events that every recursive solve uses (host-side
+ *     driver objects, no device buffers; see the conventions above).  Make both first calls
+ *     before any stream capture.
  *   - All calls share the one array and each call re-initialises what it reads; calls whose
  *     executions overlap on the same GPU (different streams, threads) race on it.
  * --------------------------------------------------------------------------------------- */

@@ -88,3 +88,13 @@ def test_clock_summary_without_samples(tmp_path):
     s = bench.ClockSampler("0")
     s.path = str(tmp_path / "missing.csv")
     assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+
+def test_prepare_flops_count_cholesky_and_inverse():
+    # a Cholesky of a k x k matrix costs sum_j (k - j - 1)(k - j) ~ k^3/3 FLOP, the triangular
+    # inverse as much again; the bench counts 2/3 k^3 per factor
+    k = 4096
+    chol = sum(2 * (k - j - 1) * (k - j) // 2 + (k - j - 1) for j in range(k))
+    assert chol == pytest.approx(k ** 3 / 3, rel=1e-3)
+    assert bench._prepare_flops(k, k) == pytest.approx(2 * 2 * k ** 3 / 3, rel=1e-12)
+    assert bench._prepare_flops(4096, 14336) == pytest.approx(2 / 3 * (4096 ** 3 + 14336 ** 3), rel=1e-12)

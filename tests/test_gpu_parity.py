@@ -4,8 +4,11 @@ Bars (stated for the two-sided GPTQ solver):
   * fp64 path: codes identical to the oracle's except at entries whose pre-rounding value
     lies within 1e-9 grid steps of a half-integer (absorbed and counted by
     oracle.compare_with_oracle); proxy loss within 1e-9 relative.
-  * fp32 path (3xTF32-class accuracy): >= 99.5 % of codes equal to the fp64 oracle's,
-    proxy loss within 1e-3 relative.
+  * fp32 path (3xTF32-class accuracy): on layers the oracle finishes (and on the leading
+    blocks of the large ones) >= 99.5 % of codes equal to the fp64 oracle's; at full size the
+    certificate, >= 99.5 % equal codes on the leading 1024 x 1024 block and the proxy loss within
+    FP32_LOSS_BAR of the fp64 path's -- a bar set from a perturbation control (see the comment
+    above test_full_size_fp32_vs_fp64_and_certificate).
 Both sides always quantize identical inputs: the factors come from the oracle side (LAPACK
 prepare) and are rounded to the solve dtype before either side sees them.
 Full-size cases are checked on the leading 256 x 256 block (which depends only on leading
@@ -210,15 +213,31 @@ def test_sq4096(kg, name, dtype):
     _leading_block_and_certificate(kg, workload(name)[0], dtype)
 
 
+# The fp32 bar at full size, set from a perturbation control (the reading is stated with its
+# numbers in the design notes).  Two-sided GPTQ is a sequence of m*n rounding decisions in which
+# one flipped decision changes every later entry to its bottom-right ("FastKron" Section 2.3), so
+# the codes of two exact solves drift apart as soon as the inputs differ at all.  The control ran
+# the fp64 path on W perturbed by delta * s_i * N(0,1) with delta = 1e-8, 1e-7 and 1e-6 grid steps
+# (3 seeds each, sq4096, ffn_up and ffn_down): at delta = 1e-7 -- some 30x below the fp32 path's own
+# median noise on the value it rounds, 3e-6 grid steps -- only 71-81 % of all codes stayed equal,
+# every leading 1024 x 1024 block kept >= 99.6 %, and the proxy loss moved by up to 2.3e-3 relative
+# (RMS 1.1e-3 over the 18 runs at delta = 1e-7 and 1e-6).  So no floating-point solve that is not
+# bit-identical to the oracle can promise 99.5 % equal codes over the whole matrix, and a loss bar of
+# 1e-3 lies inside the problem's own spread.  The fp32 bar is therefore: the certificate of the
+# fp32 solution; >= 99.5 % equal codes on the leading 1024 x 1024 block (the control's minimum);
+# and a proxy loss within FP32_LOSS_BAR = 4.5 control RMS of the fp64 loss.  The test re-runs two
+# control perturbations (delta = 1e-7) and reports them beside the fp32 figures.
+FP32_LOSS_BAR = 5e-3
+CONTROL_DELTA = 1e-7
+
+
 @pytest.mark.parametrize("name", ["sq4096", "ffn_up", "ffn_down"])
 def test_full_size_fp32_vs_fp64_and_certificate(kg, name):
     """Full-size layers: no quartic oracle at this size.  Both paths quantize identical
     (fp32-rounded) inputs.  Checked: the certificate of each path on sampled rows; the leading
-    1024 x 1024 block of codes, which depends only on leading data ("FastKron" Section 2.3) and
-    is visited before fp32 rounding has had many chances to move a value across a tie, agrees on
-    >= 99.5 %; and the proxy loss of the fp32 solution (fp64 loss kernel) is close to the fp64
-    one.  Over the whole matrix the two paths are not expected to agree code for code: every
-    tie flipped by fp32 rounding changes the entries to its bottom-right."""
+    1024 x 1024 block of codes agrees on >= 99.5 %; the proxy loss of the fp32 solution (fp64 loss
+    kernel) is within FP32_LOSS_BAR of the fp64 one.  Full-matrix agreement and the loss deviation
+    are reported next to the same figures for two fp64 solves of W perturbed by 1e-7 grid steps."""
     spec = workload(name)[0]
     W, A, B = layer_inputs(spec, device="cuda")
     UA, UB, UA32, UB32 = kg.kron_gptq_prepare(A, B, DAMP)
@@ -228,11 +247,29 @@ def test_full_size_fp32_vs_fp64_and_certificate(kg, name):
     W64, UA64, UB64, s64 = W32.double(), UA32.double(), UB32.double(), s32.double()
     c64, V64, E64 = kg.kron_gptq_quantize(W64, UA64, UB64, spec.qmin, spec.qmax, s64, want_E=True)
     k = 1024
-    agree = (c32[:k, :k] == c64[:k, :k]).float().mean().item()
-    assert agree >= 0.995, agree
+    agree_lead = (c32[:k, :k] == c64[:k, :k]).float().mean().item()
+    agree_full = (c32 == c64).float().mean().item()
     l64 = kg.kron_gptq_loss(W64, V64, A, B, DAMP)
     l32 = kg.kron_gptq_loss(W64, V32.double(), A, B, DAMP)
-    assert abs(l32 - l64) <= 1e-2 * l64, (l32, l64)
+    rel32 = (l32 - l64) / l64
+    control = []
+    for seed in (100, 101):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed)
+        Wp = W64 + CONTROL_DELTA * s64[:, None] * torch.randn(W64.shape, generator=g, device="cuda",
+                                                             dtype=torch.float64)
+        cp, Vp, _ = kg.kron_gptq_quantize(Wp, UA64, UB64, spec.qmin, spec.qmax, s64)
+        lp = kg.kron_gptq_loss(W64, Vp, A, B, DAMP)
+        control.append({"agree_full": round((cp == c64).float().mean().item(), 4),
+                        "agree_lead": round((cp[:k, :k] == c64[:k, :k]).float().mean().item(), 4),
+                        "loss_rel": float(f"{(lp - l64) / l64:.3e}")})
+        del Wp, cp, Vp
+    report = {"layer": name, "fp32_agree_full": round(agree_full, 4), "fp32_agree_lead1024": round(agree_lead, 4),
+              "fp32_loss_rel": float(f"{rel32:.3e}"), "fp64_loss": l64,
+              f"fp64_control_delta{CONTROL_DELTA:g}": control}
+    print(report)
+    assert agree_lead >= 0.995, report
+    assert abs(rel32) <= FP32_LOSS_BAR, report
     rows = np.unique(np.linspace(0, spec.m - 1, 6).astype(int))
     args = (W64.cpu().numpy(), UA64.cpu().numpy(), UB64.cpu().numpy(), s64.cpu().numpy(), spec.qmin, spec.qmax)
     cert = oracle.certificate(*args, c64.cpu().numpy(), V64.cpu().numpy(), E64.cpu().numpy(), rows=rows)
@@ -240,6 +277,27 @@ def test_full_size_fp32_vs_fp64_and_certificate(kg, name):
     cert32 = oracle.certificate(*args, c32.cpu().numpy(), V32.double().cpu().numpy(), E32.double().cpu().numpy(),
                                 rows=rows, tol=1e-4)
     assert cert32["resid_rel"] < 1e-4 and cert32["code_mismatch"] <= 1e-3 * len(rows) * spec.n, cert32
+
+
+def test_fp64_perturbation_control(kg):
+    """The control behind the fp32 bar, on the 4096 x 4096 layer: exact (fp64) solves of W and of W
+    perturbed by 1e-7 grid steps keep the leading 256 x 256 block of codes unchanged (it sees few
+    decisions before it) but differ on more than 5 % of all codes, because each flipped decision
+    changes the entries to its bottom-right ("FastKron" Section 2.3)."""
+    spec = workload("sq4096")[0]
+    W, A, B = layer_inputs(spec, device="cuda")
+    UA, UB, _, _ = kg.kron_gptq_prepare(A, B, DAMP)
+    s = kg.kron_gptq_row_scales(W, spec.qmax)
+    c0, _, _ = kg.kron_gptq_quantize(W, UA, UB, spec.qmin, spec.qmax, s)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(102)
+    Wp = W + CONTROL_DELTA * s[:, None] * torch.randn(W.shape, generator=g, device="cuda", dtype=torch.float64)
+    cp, _, _ = kg.kron_gptq_quantize(Wp, UA, UB, spec.qmin, spec.qmax, s)
+    lead = (cp[:256, :256] == c0[:256, :256]).float().mean().item()
+    full = (cp == c0).float().mean().item()
+    print({"control_lead256": lead, "control_full": full})
+    assert lead == 1.0, lead
+    assert full < 0.95, full
 
 
 # ------------------------------------------------------------------------------ edge cases, errors

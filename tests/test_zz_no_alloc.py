@@ -5,7 +5,9 @@ allocator owns the device memory, or a service path that must not call cudaMallo
 start-up.  It runs the same kernels as kron_gptq_quantize but keeps its scratch in a fixed
 device array inside the library, so its output must match the workspace entry point's
 exactly (same kernels, same launch shapes, same inputs), on two calls in a row (the second
-call finds the first call's leftovers in the shared array and must not be affected by them).
+call finds the first call's leftovers in the shared array and must not be affected by them),
+the second one on a stream of its own, and the device's free memory must not change across
+them.
 
 This file is collected last on purpose, so a failure here cannot hide other failures in a
 run that stops at the first one.
@@ -44,17 +46,31 @@ def test_noalloc_matches_workspace_entry_point(kg, dtype, m, n):
     UBt = torch.from_numpy(UB.astype(npd)).cuda()
     st = kg.kron_gptq_row_scales(Wt, spec.qmax)
     ref_codes, ref_V, ref_E = kg.kron_gptq_quantize(Wt, UAt, UBt, spec.qmin, spec.qmax, st, want_E=True)
-    for _ in range(2):
-        codes = torch.full((m, n), 99, dtype=torch.int8, device="cuda")
-        V = torch.full((m, n), float("nan"), dtype=dtype, device="cuda")
-        E = torch.full((m, n), float("nan"), dtype=dtype, device="cuda")
-        status = torch.full((1,), -99, dtype=torch.int32, device="cuda")
-        kg.kron_gptq_quantize_noalloc(Wt, UAt, UBt, spec.qmin, spec.qmax, st, codes, V, E, status)
+    outs = [(torch.empty((m, n), dtype=torch.int8, device="cuda"), torch.empty((m, n), dtype=dtype, device="cuda"),
+             torch.empty((m, n), dtype=dtype, device="cuda"), torch.empty((1,), dtype=torch.int32, device="cuda"))
+            for _ in range(2)]
+    side = torch.cuda.Stream()
+    # a warm-up call loads the kernels and creates the library's per-thread streams and events
+    kg.kron_gptq_quantize_noalloc(Wt, UAt, UBt, spec.qmin, spec.qmax, st, *outs[0])
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for k, (codes, V, E, status) in enumerate(outs):
+        codes.fill_(99)
+        V.fill_(float("nan"))
+        E.fill_(float("nan"))
+        status.fill_(-99)
+        # the second call runs on a stream of its own, after the first
+        stream = side if k == 1 else None
+        if stream is not None:
+            stream.wait_stream(torch.cuda.current_stream())
+        kg.kron_gptq_quantize_noalloc(Wt, UAt, UBt, spec.qmin, spec.qmax, st, codes, V, E, status, stream=stream)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         assert torch.equal(codes, ref_codes)
         assert torch.equal(V, ref_V)
         assert torch.equal(E, ref_E)
+    # nothing was allocated on the device by the two calls
+    assert torch.cuda.mem_get_info()[0] == free_before
 
 
 def test_noalloc_rejects_oversize_before_launch(kg):

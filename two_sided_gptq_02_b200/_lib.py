@@ -116,6 +116,9 @@ def _stream(stream):
 
 
 def _check_dev(*ts):
+    """Every tensor on the current CUDA device and contiguous: the library launches on the current
+    device and takes bare pointers, so a tensor elsewhere would be read through a wrong address."""
+    dev = None
     for t in ts:
         if t is None:
             continue
@@ -123,6 +126,40 @@ def _check_dev(*ts):
             raise ValueError("tensors must live on a CUDA device")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous (row-major)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices ({dev} and {t.device})")
+    if dev is not None and dev.index is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"tensors live on {dev} but the current device is cuda:{torch.cuda.current_device()}; "
+                         "call under torch.cuda.device(...)")
+
+
+def _check_tensor(name: str, t, dtype: torch.dtype, shape: tuple) -> None:
+    """dtype and shape of one argument; the kernels index by the sizes passed beside the pointers."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_solve_args(W, U_A, U_B, row_scale, dtype=None) -> tuple[int, int]:
+    """W (m, n), U_A (n, n), U_B (m, m) (skipped when None), row_scale (m,), all of W's dtype
+    (or `dtype`).  Returns (m, n)."""
+    if W.dim() != 2:
+        raise ValueError(f"W must be a matrix, got shape {tuple(W.shape)}")
+    m, n = W.shape
+    dtype = W.dtype if dtype is None else dtype
+    if dtype not in (torch.float32, torch.float64):
+        raise TypeError(f"unsupported dtype {dtype} (float32 or float64)")
+    _check_tensor("W", W, dtype, (m, n))
+    _check_tensor("U_A", U_A, dtype, (n, n))
+    if U_B is not None:
+        _check_tensor("U_B", U_B, dtype, (m, m))
+    _check_tensor("row_scale", row_scale, dtype, (m,))
+    return int(m), int(n)
 
 
 def _raise(rc: int, where: str):
@@ -171,12 +208,17 @@ def kron_gptq_prepare(A: torch.Tensor, B: torch.Tensor | None, damp: float, *, f
 
     Returns (U_A, U_B, U_A32, U_B32); U_B* are None when B is None.
     """
-    L = load_library()
-    _check_dev(A, B)
-    n = A.shape[0]
-    m = B.shape[0] if B is not None else 0
+    if A.dtype not in (torch.float32, torch.float64):
+        raise TypeError(f"unsupported dtype {A.dtype} (float32 or float64)")
     if B is not None and B.dtype != A.dtype:
         raise TypeError("A and B must share a dtype")
+    n = A.shape[0]
+    m = B.shape[0] if B is not None else 0
+    _check_tensor("A", A, A.dtype, (n, n))
+    if B is not None:
+        _check_tensor("B", B, A.dtype, (m, m))
+    _check_dev(A, B)
+    L = load_library()
     dev = A.device
     UA = torch.empty(n, n, dtype=torch.float64, device=dev)
     UB = torch.empty(m, m, dtype=torch.float64, device=dev) if B is not None else None
@@ -210,14 +252,11 @@ class Quantizer:
 
     def run(self, W, U_A, U_B, row_scale, qmin: int, qmax: int, stream=None) -> None:
         """Enqueue one solve on `stream`; does not synchronize."""
+        if _check_solve_args(W, U_A, U_B, row_scale, self.dtype) != (self.m, self.n):
+            raise ValueError(f"W must have shape {(self.m, self.n)}, got {tuple(W.shape)}")
+        _check_tensor("U_B", U_B, self.dtype, (self.m, self.m))
+        _check_dev(W, U_A, U_B, row_scale, self.codes)
         L = load_library()
-        for t in (W, U_A, U_B, row_scale):
-            if t.dtype != self.dtype:
-                raise TypeError("W, U_A, U_B and row_scale must all have the solve dtype")
-        _check_dev(W, U_A, U_B, row_scale)
-        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or U_B.shape != (self.m, self.m) \
-                or row_scale.shape != (self.m,):
-            raise ValueError("shape mismatch")
         grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
         rc = L.kron_gptq_quantize(_ptr(W), self.m, self.n, self.code, _ptr(U_A), _ptr(U_B), grid,
                                   _ptr(self.codes), _ptr(self.V), _ptr(self.E), _ptr(self.ws), self.ws.numel(),
@@ -243,9 +282,16 @@ def kron_gptq_quantize_noalloc(W, U_A, U_B, qmin: int, qmax: int, row_scale, cod
     """Allocation-free solve into caller-provided outputs (codes int8, V, optional E, optional
     one-int device status).  The library uses its fixed internal scratch array instead of a
     workspace; see include/kron_gptq.h for the size limit and the sharing rules."""
-    L = load_library()
+    m, n = _check_solve_args(W, U_A, U_B, row_scale)
+    _check_tensor("U_B", U_B, W.dtype, (m, m))
+    _check_tensor("codes", codes, torch.int8, (m, n))
+    _check_tensor("V", V, W.dtype, (m, n))
+    if E is not None:
+        _check_tensor("E", E, W.dtype, (m, n))
+    if dev_status is not None and (dev_status.dtype != torch.int32 or dev_status.numel() < 1):
+        raise TypeError("dev_status must be an int32 tensor with at least one element")
     _check_dev(W, U_A, U_B, row_scale, codes, V, E, dev_status)
-    m, n = W.shape
+    L = load_library()
     grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
     rc = L.kron_gptq_quantize_noalloc(_ptr(W), m, n, _dtype_code(W), _ptr(U_A), _ptr(U_B), grid, _ptr(codes),
                                       _ptr(V), _ptr(E), _ptr(dev_status), _stream(stream))
@@ -254,9 +300,16 @@ def kron_gptq_quantize_noalloc(W, U_A, U_B, qmin: int, qmax: int, row_scale, cod
 
 def kron_gptq_loss(W, V, A, B, damp: float, *, stream=None) -> float:
     """tr((V-W) A_d (V-W)^T B_d) with A_d, B_d damped as in prepare (fp64 accumulation)."""
-    L = load_library()
-    _check_dev(W, V, A, B)
+    if W.dim() != 2:
+        raise ValueError(f"W must be a matrix, got shape {tuple(W.shape)}")
     m, n = W.shape
+    _check_tensor("V", V, W.dtype, (m, n))
+    if A.dtype not in (torch.float32, torch.float64):
+        raise TypeError(f"unsupported factor dtype {A.dtype}")
+    _check_tensor("A", A, A.dtype, (n, n))
+    _check_tensor("B", B, A.dtype, (m, m))
+    _check_dev(W, V, A, B)
+    L = load_library()
     out = torch.zeros(1, dtype=torch.float64, device=W.device)
     ws = _workspace(L.kron_gptq_loss_workspace_size(m, n), W.device)
     rc = L.kron_gptq_loss(_ptr(W), _ptr(V), m, n, _dtype_code(W), _ptr(A), _ptr(B), _dtype_code(A), float(damp),
@@ -267,8 +320,10 @@ def kron_gptq_loss(W, V, A, B, damp: float, *, stream=None) -> float:
 
 
 def kron_gptq_row_scales(W, qmax: int, *, stream=None):
-    L = load_library()
+    if W.dim() != 2:
+        raise ValueError(f"W must be a matrix, got shape {tuple(W.shape)}")
     _check_dev(W)
+    L = load_library()
     m, n = W.shape
     s = torch.empty(m, dtype=W.dtype, device=W.device)
     _raise(L.kron_gptq_row_scales(_ptr(W), m, n, _dtype_code(W), int(qmax), _ptr(s), _stream(stream)),
@@ -291,14 +346,12 @@ class RcQuantizer:
 
     def run(self, W, U_A, U_B, alpha, beta, stream=None) -> None:
         """Enqueue one solve on `stream`; does not synchronize."""
+        if _check_solve_args(W, U_A, U_B, beta, self.dtype) != (self.m, self.n):
+            raise ValueError(f"W must have shape {(self.m, self.n)}, got {tuple(W.shape)}")
+        _check_tensor("U_B", U_B, self.dtype, (self.m, self.m))
+        _check_tensor("alpha", alpha, self.dtype, (self.n,))
+        _check_dev(W, U_A, U_B, alpha, beta, self.Z)
         L = load_library()
-        for t in (W, U_A, U_B, alpha, beta):
-            if t.dtype != self.dtype:
-                raise TypeError("W, U_A, U_B, alpha and beta must all have the solve dtype")
-        _check_dev(W, U_A, U_B, alpha, beta)
-        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or U_B.shape != (self.m, self.m) \
-                or alpha.shape != (self.n,) or beta.shape != (self.m,):
-            raise ValueError("shape mismatch")
         rc = L.kron_gptq_quantize_rc(_ptr(W), self.m, self.n, self.code, _ptr(U_A), _ptr(U_B), _ptr(alpha),
                                      _ptr(beta), _ptr(self.Z), _ptr(self.V), _ptr(self.E), _ptr(self.ws),
                                      self.ws.numel(), _stream(stream))
@@ -320,11 +373,13 @@ def kron_gptq_quantize_rc(W, U_A, U_B, alpha, beta, *, want_E: bool = False, str
 
 def kron_gptq_waterkron_scales(U_A, U_B, gamma: float, *, stream=None):
     """WaterKron steps: alpha = sqrt(gamma) diag(U_A), beta = sqrt(gamma) diag(U_B)."""
-    L = load_library()
-    _check_dev(U_A, U_B)
     if U_A.dtype != U_B.dtype:
         raise TypeError("U_A and U_B must share a dtype")
     n, m = U_A.shape[0], U_B.shape[0]
+    _check_tensor("U_A", U_A, U_A.dtype, (n, n))
+    _check_tensor("U_B", U_B, U_A.dtype, (m, m))
+    _check_dev(U_A, U_B)
+    L = load_library()
     alpha = torch.empty(n, dtype=U_A.dtype, device=U_A.device)
     beta = torch.empty(m, dtype=U_B.dtype, device=U_B.device)
     _raise(L.kron_gptq_waterkron_scales(_ptr(U_A), n, _ptr(U_B), m, _dtype_code(U_A), float(gamma), _ptr(alpha),
@@ -363,13 +418,10 @@ class OnesidedQuantizer:
         self.E = torch.empty(self.m, self.n, dtype=dtype, device=device) if want_E else None
 
     def run(self, W, U_A, row_scale, qmin: int, qmax: int, stream=None) -> None:
+        if _check_solve_args(W, U_A, None, row_scale, self.dtype) != (self.m, self.n):
+            raise ValueError(f"W must have shape {(self.m, self.n)}, got {tuple(W.shape)}")
+        _check_dev(W, U_A, row_scale, self.codes)
         L = load_library()
-        for t in (W, U_A, row_scale):
-            if t.dtype != self.dtype:
-                raise TypeError("W, U_A and row_scale must all have the solve dtype")
-        _check_dev(W, U_A, row_scale)
-        if W.shape != (self.m, self.n) or U_A.shape != (self.n, self.n) or row_scale.shape != (self.m,):
-            raise ValueError("shape mismatch")
         grid = _Grid(int(qmin), int(qmax), row_scale.data_ptr())
         rc = L.kron_gptq_quantize_onesided(_ptr(W), self.m, self.n, self.code, _ptr(U_A), grid, _ptr(self.codes),
                                            _ptr(self.V), _ptr(self.E), _ptr(self.ws), self.ws.numel(),
@@ -396,14 +448,20 @@ FACTOR_METHODS = {"marginal": 0, "frobenius": 1, "flipflop": 2}
 def kron_gptq_factors(a, b, method: str = "flipflop", iters: int = 2, *, stream=None, check: bool = True):
     """Kronecker factors (A n x n, B m x m, fp64) of E[a a^T (x) b b^T] from samples a (N x n) and
     b (N x m): "marginal", "frobenius" or "flipflop" (iters alternating updates from B = I)."""
-    L = load_library()
-    _check_dev(a, b)
     if a.dtype != b.dtype:
         raise TypeError("a and b must share a dtype")
+    if a.dtype not in (torch.float32, torch.float64):
+        raise TypeError(f"unsupported dtype {a.dtype} (float32 or float64)")
+    if a.dim() != 2 or b.dim() != 2:
+        raise ValueError("a and b must be matrices (samples x channels)")
     N, n = a.shape
     if b.shape[0] != N:
         raise ValueError("a and b need the same number of samples")
     m = b.shape[1]
+    if method not in FACTOR_METHODS:
+        raise ValueError(f"method must be one of {sorted(FACTOR_METHODS)}")
+    _check_dev(a, b)
+    L = load_library()
     A = torch.empty(n, n, dtype=torch.float64, device=a.device)
     B = torch.empty(m, m, dtype=torch.float64, device=a.device)
     ws = _workspace(L.kron_gptq_factors_workspace_size(N, n, m), a.device)
@@ -419,11 +477,12 @@ def kron_gptq_quantize_antidiagonal(W, U_A, U_B, qmin: int, qmax: int, row_scale
                                     stream=None, check: bool = True):
     """The non-recursive anti-diagonal baseline (quartic work; fp64).  Same outputs as
     kron_gptq_quantize: (codes int8, V, E or None)."""
-    L = load_library()
-    _check_dev(W, U_A, U_B, row_scale)
     if W.dtype != torch.float64:
         raise TypeError("the anti-diagonal baseline runs in fp64")
-    m, n = W.shape
+    m, n = _check_solve_args(W, U_A, U_B, row_scale)
+    _check_tensor("U_B", U_B, W.dtype, (m, m))
+    _check_dev(W, U_A, U_B, row_scale)
+    L = load_library()
     ws = _workspace(L.kron_gptq_quantize_antidiagonal_workspace_size(m, n), W.device)
     codes = torch.empty(m, n, dtype=torch.int8, device=W.device)
     V = torch.empty(m, n, dtype=W.dtype, device=W.device)

@@ -43,7 +43,18 @@ constexpr int WS_RING = 8;                                   // slots of the (P,
 constexpr int WS_GROUPS = 2;                                 // helper groups, alternating steps
 constexpr int WS_HELPERS = 256 * WS_GROUPS;                  // eight warps per group
 constexpr int WS_THREADS = WS_HELPERS + 32;                  // + the rounding warp
+#ifndef KG_TEST_HANDOFF_FAULT
 constexpr long long WS_MAX_WAIT_CYCLES = 50000000LL;         // ~25 ms: far beyond any hand-off
+#else
+// Test build only (python -m two_sided_gptq_02_b200.build --define KG_TEST_HANDOFF_FAULT --out ...):
+// a shorter limit, and a device switch that makes the helpers of row 0 in the first leaf (tile
+// anti-diagonal 0) withhold their arrival for step 5, so that the rounding warp's bounded wait on
+// that slot runs out.  The wait then gives up, the CTA raises its abort flag, every other wait of
+// the CTA ends at its next check of the flag, and the leaf records KG_ERR_TIMEOUT and returns.
+// Nothing faults or traps: the kernel only skips work.  The default build contains none of this.
+constexpr long long WS_MAX_WAIT_CYCLES = 4000000LL;          // ~2 ms
+__device__ int g_test_handoff_fault;
+#endif
 
 struct LeafWsSmem {
     static constexpr int S = LeafCfg<float>::S;
@@ -371,7 +382,12 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                 sm.pre[d % WS_RING][i][0] = w - c;
                 sm.pre[d % WS_RING][i][1] = r;
             }
-            if (q == 0) tc::mbar_arrive(&sm.hbar[d % WS_RING]);
+#ifdef KG_TEST_HANDOFF_FAULT
+            const bool withhold = g_test_handoff_fault != 0 && D == 0 && i == 0 && d == 5;
+#else
+            constexpr bool withhold = false;
+#endif
+            if (q == 0 && !withhold) tc::mbar_arrive(&sm.hbar[d % WS_RING]);
         }
     }
     if (!ok) {

@@ -35,9 +35,6 @@
 #include "kg_gemm.cuh"
 #include "kg_leaf.cuh"
 #include "kg_leaf_ws.cuh"
-#ifdef KG_EXPERIMENTAL_PAIR
-#include "kg_leaf_pair.cuh"
-#endif
 #include "kg_profile.cuh"
 #include "kg_push_tc.cuh"
 #include "kg_rc.cuh"
@@ -60,9 +57,6 @@ struct QLayout {
     size_t es;
     size_t off_wt, off_r, off_e, off_s, off_ua, off_ub;
     size_t off_elo, off_uat, off_uatlo, off_ubt, off_ubtlo, off_xt, off_xtlo, total;
-#ifdef KG_EXPERIMENTAL_PAIR
-    size_t off_sync, sync_bytes;
-#endif
 };
 
 static QLayout q_layout(int64_t m, int64_t n, size_t es) {
@@ -96,12 +90,6 @@ static QLayout q_layout(int64_t m, int64_t n, size_t es) {
         plane(L.off_ubtlo, L.Mp * L.Mp);
         plane(L.off_xt, L.Np * L.Mp);
         plane(L.off_xtlo, L.Np * L.Mp);
-#ifdef KG_EXPERIMENTAL_PAIR
-        // paired leaves: one ticket counter per tile anti-diagonal, one progress word per tile row
-        L.off_sync = off;
-        L.sync_bytes = align_up((size_t)(L.Mt + L.Nt - 1 + L.Mt) * sizeof(int), 256);
-        off += L.sync_bytes;
-#endif
     }
     L.total = off;
     return L;
@@ -224,11 +212,6 @@ struct QArgs {
     Real *Elo, *XT, *XTlo, *UAT, *UATlo, *UBT, *UBTlo;
     // their tensor maps (fp32 only)
     const PushTmaMaps* maps;
-#ifdef KG_EXPERIMENTAL_PAIR
-    // paired leaves (fp32 only): ticket counters per tile anti-diagonal, progress words per tile row
-    int* tickets;
-    int* prog;
-#endif
 };
 
 // Launch with programmatic stream serialization when pdl is set: the kernel may start while the
@@ -266,17 +249,6 @@ static int launch_leaf(const QArgs<Real>& a, int D, cudaStream_t st) {
     }
 }
 
-#ifdef KG_EXPERIMENTAL_PAIR
-// Tile anti-diagonals D and D+1 in one launch (fp32): the update from D to D+1 happens inside.
-static int launch_pair(const QArgs<float>& a, int D, cudaStream_t st) {
-    const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    auto count = [&](int d) { return std::min(d, Mt - 1) - std::max(0, d - Nt + 1) + 1; };
-    ProfScope ps(PK_LEAF, st);
-    return launch_k(k_leaf_pair, dim3(count(D) + count(D + 1)), dim3(PAIR_THREADS), sizeof(LeafPairSmem), st, true,
-                    D, Mt, Nt, a.L.m, a.L.n, a.L.Np, a.L.Mp, a.Wt, a.R, a.E, a.Elo, a.XT, a.XTlo, a.UA, a.ldA, a.UB,
-                    a.ldB, a.sp, a.qmin, a.qmax, a.codes, a.code_bytes, a.V, a.outE, a.status, a.tickets + D, a.prog);
-}
-#endif
 
 // Update of the targets on diagonals [tgt0, D1) from the sources on diagonals [D0, mid).
 static int launch_push(const QArgs<double>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st, bool pdl) {
@@ -344,14 +316,6 @@ static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
         if ((rc = sched_wait(s, D0, D0 + 1))) return rc;
         return launch_leaf(a, D0, s.crit);
     }
-#ifdef KG_EXPERIMENTAL_PAIR
-    if constexpr (sizeof(Real) == 4) {
-        if (D1 - D0 == 2) {   // two diagonals: one paired launch, no update between them
-            if ((rc = sched_wait(s, D0, D1))) return rc;
-            return launch_pair(a, D0, s.crit);
-        }
-    }
-#endif
     const int mid = (D0 + D1) / 2;
     if ((rc = solve_range(a, s, D0, mid))) return rc;
     if ((rc = sched_wait(s, mid, mid + 1))) return rc;
@@ -490,9 +454,6 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
     }
     a.Elo = a.XT = a.XTlo = a.UAT = a.UATlo = a.UBT = a.UBTlo = nullptr;
     a.maps = nullptr;
-#ifdef KG_EXPERIMENTAL_PAIR
-    a.tickets = a.prog = nullptr;
-#endif
     PushTmaMaps maps;
     if (sizeof(Real) == 4) {
         a.Elo = reinterpret_cast<Real*>(base + L.off_elo);
@@ -502,11 +463,6 @@ static int quantize_impl(const void* W, int64_t m, int64_t n, const void* UA_, c
         a.UBTlo = reinterpret_cast<Real*>(base + L.off_ubtlo);
         a.XT = reinterpret_cast<Real*>(base + L.off_xt);
         a.XTlo = reinterpret_cast<Real*>(base + L.off_xtlo);
-#ifdef KG_EXPERIMENTAL_PAIR
-        a.tickets = reinterpret_cast<int*>(base + L.off_sync);
-        a.prog = a.tickets + (L.Mt + L.Nt - 1);
-        KG_CUDA_TRY(cudaMemsetAsync(base + L.off_sync, 0, L.sync_bytes, st));
-#endif
         const SplitOperands op{reinterpret_cast<const float*>(a.E), reinterpret_cast<const float*>(a.Elo),
                                reinterpret_cast<const float*>(a.XT), reinterpret_cast<const float*>(a.XTlo),
                                reinterpret_cast<const float*>(a.UAT), reinterpret_cast<const float*>(a.UATlo),
@@ -550,12 +506,6 @@ static int configure_leaf() {
                                              (int)sizeof(LeafWsSmem)));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_ws, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
-#ifdef KG_EXPERIMENTAL_PAIR
-            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)sizeof(LeafPairSmem)));
-            KG_CUDA_TRY(cudaFuncSetAttribute(k_leaf_pair, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                             cudaSharedmemCarveoutMaxShared));
-#endif
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              PushCfg<1>::SMEM_BYTES));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -912,14 +862,12 @@ extern "C" int kron_gptq_quantize_antidiagonal(const void* W, int64_t m, int64_t
                                  static_cast<unsigned char*>(ws) + qbytes);
 }
 
-#ifdef KG_PAIR_TIMELINE
-// Copies the paired launches' per-CTA timeline (kg_leaf_pair.cuh) to host memory: count words at
-// most.  0 on success, KG_ERR_CUDA otherwise.  Only in builds with KG_PAIR_TIMELINE.
-extern "C" __attribute__((visibility("default"))) int kron_gptq_debug_pair_timeline(unsigned long long* host,
-                                                                                    size_t count) {
-    count = std::min(count, sizeof(kg::g_pair_tl) / sizeof(unsigned long long));
-    if (cudaMemcpyFromSymbol(host, kg::g_pair_tl, count * sizeof(unsigned long long)) != cudaSuccess)
-        return KG_ERR_CUDA;
-    return 0;
+#ifdef KG_TEST_HANDOFF_FAULT
+// Test build only: switch the withheld hand-off of kg_leaf_ws.cuh on (1) or off (0) on the
+// current device.  0 on success, KG_ERR_CUDA otherwise.  Not part of the C ABI of the default
+// library, which does not contain it.
+extern "C" __attribute__((visibility("default"))) int kron_gptq_debug_handoff_fault(int on) {
+    const int v = on ? 1 : 0;
+    return cudaMemcpyToSymbol(kg::g_test_handoff_fault, &v, sizeof(v)) == cudaSuccess ? 0 : KG_ERR_CUDA;
 }
 #endif
