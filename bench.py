@@ -258,8 +258,8 @@ def _onesided(kg, torch, spec, Wd, UAd, sd, steps, solve_ms):
             "leaf_ms": prof["leaf"][1], "leaf_launches": prof["leaf"][0], "gemm_ms": prof["push"][1],
             "gemm_launches": prof["push"][0],
             "gemm_flops": float(m) * n * n, "steps": steps,
-            "note": "kron_gptq_quantize_onesided (64-column leaves + cuBLAS GEMM updates: BF16x9 in fp32, "
-                    "DGEMM in fp64) on the same W, U_A, scales and grid; inputs resident"}
+            "note": "kron_gptq_quantize_onesided (64-column leaves + the library's own tensor-core GEMM updates: "
+                    "tcgen05 3xTF32 in fp32, FP64 mma in fp64) on the same W, U_A, scales and grid; inputs resident"}
 
 
 def _factors(kg, torch, spec, fp64_peak, reps=3, iters=2, N=4096):

@@ -19,11 +19,12 @@
  *   - All matrices are dense, row-major, contiguous, in DEVICE memory owned by the caller.
  *     The library never allocates or frees device memory: each call takes a caller-owned
  *     workspace of at least the size the matching *_workspace_size() function returns.  The one
- *     exception: the calls that hand a plain dense GEMM to cuBLAS (quantize_onesided, factors,
- *     quantize_antidiagonal) create one cuBLAS handle per host thread and device on first use,
- *     and cuBLAS allocates its own small device state then; their GEMM workspace is inside ws.
+ *     exception: quantize_antidiagonal, the quartic baseline kept as a yardstick, hands its dense
+ *     products to cuBLAS; it creates one cuBLAS handle per host thread and device on first use,
+ *     and cuBLAS allocates its own small device state then (its GEMM workspace is inside ws).
  *     Handles live until the process exits, also those of threads that have ended, so make
- *     these calls from long-lived threads.
+ *     that call from long-lived threads.  Every other product runs in the library's own
+ *     kernels.
  *   - Calls are asynchronous on the given CUDA stream (passed as void*, a cudaStream_t;
  *     NULL = the legacy default stream).  Errors the host can see (bad arguments,
  *     unsupported options, a failed launch) are returned at once and nothing is launched
@@ -271,10 +272,8 @@ KG_API int kron_gptq_code_entropy(const int32_t* Z, int64_t count, double* out_b
  *       c = clamp(rint(x / s_i), qmin, qmax),  Q = s_i c,  E_ij = (x - Q) / U_A[j,j],
  *       W[i, j'] -= E_ij U_A[j, j']   for j' > j.
  *   The result equals kron_gptq_quantize with U_B = I (up to rounding ties).  The recursion stops
- *   at 64-column blocks; each batched update is a dense GEMM done by cuBLAS on the tensor cores
- *   (fp32: BF16x9 emulation of fp32; fp64: DGEMM), with its workspace inside ws.  cuBLAS keeps one
- *   handle per host thread and device, created on the first call (cublasCreate allocates its own
- *   small device state then; nothing else is allocated).
+ *   at 64-column blocks; each batched update is one dense GEMM on the tensor cores in the
+ *   library's own kernels (fp32: tcgen05 with 3xTF32 split operands; fp64: the FP64 mma path).
  * Arguments: W (m x n), U_A (n x n, 16-byte aligned), grid, out_codes (int8), out_V, out_E
  *   (optional): as kron_gptq_quantize.  ws: kron_gptq_quantize_onesided_workspace_size(m, n, dtype) bytes,
  *   256-byte aligned, status word first.
@@ -298,7 +297,7 @@ KG_API int kron_gptq_quantize_onesided(const void* W, int64_t m, int64_t n, int 
  *     KG_FACTOR_FLIPFLOP:  from B = I, repeat: A = E[(b^T B^-1 b) a a^T] / m,
  *                          B = E[(a^T A^-1 a) b b^T] / n.
  *   iters (>= 1) is the number of (A, B) updates of the two alternating methods.  Computed in
- *   fp64: DGEMMs (cuBLAS, workspace inside ws) and the library's own prepare for A^-1, B^-1.
+ *   fp64: the library's own DGEMMs on the FP64 tensor path and its own prepare for A^-1, B^-1.
  * Arguments:
  *   a, b      device, row-major N x n and N x m, dtype KG_F32 (promoted) or KG_F64.
  *   A, B      device fp64 outputs, n x n and m x m, symmetric.

@@ -13,23 +13,32 @@
 // Everything is fp64 and GEMM-shaped: a weighted Gram X^T diag(w) X is one GEMM of X with its
 // row-scaled copy; the weights x_k^T M x_k are one GEMM (Y = X M) and a row-wise dot; for
 // FlipFlop M^-1 = U^T U with U from kron_gptq_prepare (damping 0), so x_k^T M^-1 x_k = ||U x_k||^2.
-// The GEMMs go to cuBLAS (DGEMM), with a workspace slice of the call's workspace.
+// The GEMMs are the library's own DGEMM on the FP64 tensor path (kg_dgemm.cuh); the samples and
+// every operand are kept zero-padded to multiples of 64 in the workspace, so the padding adds
+// nothing to any product.
 #include <algorithm>
 
-#include "kg_blas.cuh"
 #include "kg_common.cuh"
+#include "kg_dgemm.cuh"
 #include "kg_profile.cuh"
 
 namespace kg {
 
-constexpr size_t FAC_BLAS_WS = 32u << 20;
+static inline int64_t pad64(int64_t x) { return ceil_div(x, 64) * 64; }
 
+// dst (rp x cp, zero padded) = src (rows x cols, row-major, any dtype promoted to fp64); with a
+// status word, non-finite input is reported
 template <typename T>
-__global__ void k_fac_copy(const T* __restrict__ src, int64_t cnt, double* __restrict__ dst, DevStatus* status) {
+__global__ void k_fac_pad(const T* __restrict__ src, int64_t rows, int64_t cols, double* __restrict__ dst,
+                          int64_t rp, int64_t cp, DevStatus* status) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < cnt; p += stride) {
-        const double v = (double)src[p];
-        if (!isfinite(v)) set_status(status, KG_ERR_NONFINITE, (int)(p < INT32_MAX ? p : INT32_MAX));
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < rp * cp; p += stride) {
+        const int64_t r = p / cp, c = p - r * cp;
+        double v = 0.0;
+        if (r < rows && c < cols) {
+            v = (double)src[r * cols + c];
+            if (status && !isfinite(v)) set_status(status, KG_ERR_NONFINITE, (int)std::min<int64_t>(r * cols + c, INT32_MAX));
+        }
         dst[p] = v;
     }
 }
@@ -59,16 +68,12 @@ __global__ void k_fac_scale_rows(const double* __restrict__ X, const double* __r
     for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < N * k; p += stride) Xw[p] = X[p] * w[p / k];
 }
 
-// M = (M + M^T) / 2
-__global__ void k_fac_sym(double* __restrict__ M, int64_t k) {
+// out (k x k) = (G + G^T) / 2 on the leading block of the padded G (ld gp)
+__global__ void k_fac_sym_out(const double* __restrict__ G, int64_t gp, double* __restrict__ out, int64_t k) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < k * k; p += stride) {
         const int64_t i = p / k, j = p - i * k;
-        if (j > i) {
-            const double v = 0.5 * (M[i * k + j] + M[j * k + i]);
-            M[i * k + j] = v;
-            M[j * k + i] = v;
-        }
+        out[p] = 0.5 * (G[i * gp + j] + G[j * gp + i]);
     }
 }
 
@@ -101,79 +106,71 @@ __global__ void k_fac_merge_status(DevStatus* dst, const DevStatus* src) {
 }
 
 struct FacLayout {
-    size_t off_a, off_b, off_y, off_xw, off_w, off_u, off_scal, off_prep, off_blas, total;
+    int64_t Np, np, mp, kp;
+    size_t off_a, off_b, off_y, off_xw, off_w, off_u, off_upad, off_g, off_scal, off_prep, total;
 };
 
 static FacLayout fac_layout(int64_t N, int64_t n, int64_t m) {
     const int64_t k = std::max(n, m);
     FacLayout L{};
+    L.Np = pad64(N); L.np = pad64(n); L.mp = pad64(m); L.kp = pad64(k);
     size_t off = kStatusBytes;
     auto take = [&](size_t& o, size_t bytes) { o = off; off = align_up(off + bytes, 256); };
-    take(L.off_a, (size_t)(N * n) * 8);
-    take(L.off_b, (size_t)(N * m) * 8);
-    take(L.off_y, (size_t)(N * k) * 8);
-    take(L.off_xw, (size_t)(N * k) * 8);
-    take(L.off_w, (size_t)N * 8);
+    take(L.off_a, (size_t)(L.Np * L.np) * 8);
+    take(L.off_b, (size_t)(L.Np * L.mp) * 8);
+    take(L.off_y, (size_t)(L.Np * L.kp) * 8);
+    take(L.off_xw, (size_t)(L.Np * L.kp) * 8);
+    take(L.off_w, (size_t)L.Np * 8);
     take(L.off_u, (size_t)(k * k) * 8);
+    take(L.off_upad, (size_t)(L.kp * L.kp) * 8);
+    take(L.off_g, (size_t)(L.kp * L.kp) * 8);
     take(L.off_scal, 256);
     take(L.off_prep, kron_gptq_prepare_workspace_size(k));
-    L.off_blas = off;
-    off += FAC_BLAS_WS;
     L.total = off;
     return L;
 }
 
 struct Fac {
-    cublasHandle_t h;
     cudaStream_t st;
     DevStatus* status;
-    double *y, *xw, *w, *u, *scal;
+    double *y, *xw, *w, *u, *upad, *g, *scal;
     void* prep;
     size_t prep_bytes;
-    int64_t N;
+    int64_t N, Np;
 };
 
 static int grid_for(int64_t cnt) { return (int)std::max<int64_t>(1, std::min<int64_t>(148 * 4, ceil_div(cnt, 256))); }
 
-// G = X^T diag(w) X (the weights carry every constant), symmetrised.  Row-major X (N x k) is
-// column-major X^T (k x N); with Xw = diag(w) X, G = X^T Xw is gemm(N, T) of the column-major
-// views X^T and Xw^T.
-static int fac_gram(const Fac& f, const double* X, int64_t k, double* G) {
-    k_fac_scale_rows<<<grid_for(f.N * k), 256, 0, f.st>>>(X, f.w, f.N, k, f.xw);
+// G (k x k) = X^T diag(w) X (the weights carry every constant), symmetrised; X is Np x px, zero padded.
+static int fac_gram(const Fac& f, const double* X, int64_t px, int64_t k, double* G) {
+    k_fac_scale_rows<<<grid_for(f.Np * px), 256, 0, f.st>>>(X, f.w, f.Np, px, f.xw);
     KG_LAUNCH_CHECK();
-    const double one = 1.0, zero = 0.0;
-    if (cublasDgemm(f.h, CUBLAS_OP_N, CUBLAS_OP_T, (int)k, (int)k, (int)f.N, &one, X, (int)k, f.xw, (int)k, &zero, G,
-                    (int)k) != CUBLAS_STATUS_SUCCESS)
-        return KG_ERR_CUDA;
-    k_fac_sym<<<grid_for(k * k), 256, 0, f.st>>>(G, k);
+    if (!dgemm(f.st, DG_TRANS_A, (int)px, (int)px, (int)f.Np, 1.0, X, px, f.xw, px, 0.0, f.g, px)) return KG_ERR_CUDA;
+    k_fac_sym_out<<<grid_for(k * k), 256, 0, f.st>>>(f.g, px, G, k);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
 
-// w_r = fh / *fd * x_r^T M x_r  (Y = X M: column-major Y^T = M^T X^T, and row-major M is
-// column-major M^T)
-static int fac_form(const Fac& f, const double* X, int64_t k, const double* M, double fh, const double* fd) {
-    const double one = 1.0, zero = 0.0;
-    if (cublasDgemm(f.h, CUBLAS_OP_N, CUBLAS_OP_N, (int)k, (int)f.N, (int)k, &one, M, (int)k, X, (int)k, &zero, f.y,
-                    (int)k) != CUBLAS_STATUS_SUCCESS)
-        return KG_ERR_CUDA;
-    k_fac_rowform<<<grid_for(f.N * 32), 256, 0, f.st>>>(f.y, X, f.N, k, 0, fh, fd, f.w);
+// w_r = fh / *fd * x_r^T M x_r with Y = X M (M k x k, padded into upad)
+static int fac_form(const Fac& f, const double* X, int64_t px, int64_t k, const double* M, double fh, const double* fd) {
+    k_fac_pad<double><<<grid_for(px * px), 256, 0, f.st>>>(M, k, k, f.upad, px, px, nullptr);
+    KG_LAUNCH_CHECK();
+    if (!dgemm(f.st, 0, (int)f.Np, (int)px, (int)px, 1.0, X, px, f.upad, px, 0.0, f.y, px)) return KG_ERR_CUDA;
+    k_fac_rowform<<<grid_for(f.Np * 32), 256, 0, f.st>>>(f.y, X, f.Np, px, 0, fh, fd, f.w);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
 
-// w_r = fh * x_r^T M^-1 x_r = fh * ||U x_r||^2 with U^T U = M^-1 (prepare, damping 0):
-// Y = X U^T, column-major Y^T = U X^T = op_T(U^T) X^T
-static int fac_form_inv(const Fac& f, const double* X, int64_t k, const double* M, double fh) {
+// w_r = fh * x_r^T M^-1 x_r = fh * ||U x_r||^2 with U^T U = M^-1 (prepare, damping 0): Y = X U^T
+static int fac_form_inv(const Fac& f, const double* X, int64_t px, int64_t k, const double* M, double fh) {
     int rc = kron_gptq_prepare(M, k, nullptr, 0, KG_F64, 0.0, f.u, nullptr, nullptr, nullptr, f.prep, f.prep_bytes, f.st);
     if (rc) return rc;
     k_fac_merge_status<<<1, 32, 0, f.st>>>(f.status, static_cast<const DevStatus*>(f.prep));
     KG_LAUNCH_CHECK();
-    const double one = 1.0, zero = 0.0;
-    if (cublasDgemm(f.h, CUBLAS_OP_T, CUBLAS_OP_N, (int)k, (int)f.N, (int)k, &one, f.u, (int)k, X, (int)k, &zero, f.y,
-                    (int)k) != CUBLAS_STATUS_SUCCESS)
-        return KG_ERR_CUDA;
-    k_fac_rowform<<<grid_for(f.N * 32), 256, 0, f.st>>>(f.y, X, f.N, k, 1, fh, nullptr, f.w);
+    k_fac_pad<double><<<grid_for(px * px), 256, 0, f.st>>>(f.u, k, k, f.upad, px, px, nullptr);
+    KG_LAUNCH_CHECK();
+    if (!dgemm(f.st, DG_TRANS_B, (int)f.Np, (int)px, (int)px, 1.0, X, px, f.upad, px, 0.0, f.y, px)) return KG_ERR_CUDA;
+    k_fac_rowform<<<grid_for(f.Np * 32), 256, 0, f.st>>>(f.y, X, f.Np, px, 1, fh, nullptr, f.w);
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
@@ -189,35 +186,34 @@ static int factors_impl(const void* a, const void* b, int64_t N, int64_t n, int6
     f.xw = reinterpret_cast<double*>(base + L.off_xw);
     f.w = reinterpret_cast<double*>(base + L.off_w);
     f.u = reinterpret_cast<double*>(base + L.off_u);
+    f.upad = reinterpret_cast<double*>(base + L.off_upad);
+    f.g = reinterpret_cast<double*>(base + L.off_g);
     f.scal = reinterpret_cast<double*>(base + L.off_scal);
     f.prep = base + L.off_prep;
-    f.prep_bytes = L.off_blas - L.off_prep;
+    f.prep_bytes = L.total - L.off_prep;
     f.N = N;
+    f.Np = L.Np;
     double* ad = reinterpret_cast<double*>(base + L.off_a);
     double* bd = reinterpret_cast<double*>(base + L.off_b);
-    int rc = blas_handle(&f.h);
-    if (!rc) rc = blas_bind(f.h, st, base + L.off_blas, FAC_BLAS_WS);
-    if (rc) return rc;
+    const int64_t np = L.np, mp = L.mp;
     KG_CUDA_TRY(cudaMemsetAsync(f.status, 0, kStatusBytes, st));
     if (dtype == KG_F64) {
-        k_fac_copy<double><<<grid_for(N * n), 256, 0, st>>>(static_cast<const double*>(a), N * n, ad, f.status);
-        k_fac_copy<double><<<grid_for(N * m), 256, 0, st>>>(static_cast<const double*>(b), N * m, bd, f.status);
+        k_fac_pad<double><<<grid_for(L.Np * np), 256, 0, st>>>(static_cast<const double*>(a), N, n, ad, L.Np, np, f.status);
+        k_fac_pad<double><<<grid_for(L.Np * mp), 256, 0, st>>>(static_cast<const double*>(b), N, m, bd, L.Np, mp, f.status);
     } else {
-        k_fac_copy<float><<<grid_for(N * n), 256, 0, st>>>(static_cast<const float*>(a), N * n, ad, f.status);
-        k_fac_copy<float><<<grid_for(N * m), 256, 0, st>>>(static_cast<const float*>(b), N * m, bd, f.status);
+        k_fac_pad<float><<<grid_for(L.Np * np), 256, 0, st>>>(static_cast<const float*>(a), N, n, ad, L.Np, np, f.status);
+        k_fac_pad<float><<<grid_for(L.Np * mp), 256, 0, st>>>(static_cast<const float*>(b), N, m, bd, L.Np, mp, f.status);
     }
     KG_LAUNCH_CHECK();
     const double invN = 1.0 / (double)N;
+    int rc;
     for (int it = 0; it < (method == KG_FACTOR_MARGINAL ? 1 : iters); ++it) {
         if (method == KG_FACTOR_MARGINAL) {
-            const double one = invN, zero = 0.0;
-            if (cublasDgemm(f.h, CUBLAS_OP_N, CUBLAS_OP_T, (int)n, (int)n, (int)N, &one, ad, (int)n, ad, (int)n, &zero, A,
-                            (int)n) != CUBLAS_STATUS_SUCCESS ||
-                cublasDgemm(f.h, CUBLAS_OP_N, CUBLAS_OP_T, (int)m, (int)m, (int)N, &one, bd, (int)m, bd, (int)m, &zero, B,
-                            (int)m) != CUBLAS_STATUS_SUCCESS)
-                return KG_ERR_CUDA;
-            k_fac_sym<<<grid_for(n * n), 256, 0, st>>>(A, n);
-            k_fac_sym<<<grid_for(m * m), 256, 0, st>>>(B, m);
+            if (!dgemm(st, DG_TRANS_A, (int)np, (int)np, (int)L.Np, invN, ad, np, ad, np, 0.0, f.g, np)) return KG_ERR_CUDA;
+            k_fac_sym_out<<<grid_for(n * n), 256, 0, st>>>(f.g, np, A, n);
+            KG_LAUNCH_CHECK();
+            if (!dgemm(st, DG_TRANS_A, (int)mp, (int)mp, (int)L.Np, invN, bd, mp, bd, mp, 0.0, f.g, mp)) return KG_ERR_CUDA;
+            k_fac_sym_out<<<grid_for(m * m), 256, 0, st>>>(f.g, mp, B, m);
             KG_LAUNCH_CHECK();
             break;
         }
@@ -228,17 +224,17 @@ static int factors_impl(const void* a, const void* b, int64_t N, int64_t n, int6
         if (method == KG_FACTOR_FROBENIUS) {
             k_fac_sumsq<<<1, 1024, 0, st>>>(B, m * m, f.scal);
             KG_LAUNCH_CHECK();
-            if ((rc = fac_form(f, bd, m, B, invN, f.scal))) return rc;
-            if ((rc = fac_gram(f, ad, n, A))) return rc;
+            if ((rc = fac_form(f, bd, mp, m, B, invN, f.scal))) return rc;
+            if ((rc = fac_gram(f, ad, np, n, A))) return rc;
             k_fac_sumsq<<<1, 1024, 0, st>>>(A, n * n, f.scal + 1);
             KG_LAUNCH_CHECK();
-            if ((rc = fac_form(f, ad, n, A, invN, f.scal + 1))) return rc;
-            if ((rc = fac_gram(f, bd, m, B))) return rc;
+            if ((rc = fac_form(f, ad, np, n, A, invN, f.scal + 1))) return rc;
+            if ((rc = fac_gram(f, bd, mp, m, B))) return rc;
         } else {
-            if ((rc = fac_form_inv(f, bd, m, B, invN / (double)m))) return rc;
-            if ((rc = fac_gram(f, ad, n, A))) return rc;
-            if ((rc = fac_form_inv(f, ad, n, A, invN / (double)n))) return rc;
-            if ((rc = fac_gram(f, bd, m, B))) return rc;
+            if ((rc = fac_form_inv(f, bd, mp, m, B, invN / (double)m))) return rc;
+            if ((rc = fac_gram(f, ad, np, n, A))) return rc;
+            if ((rc = fac_form_inv(f, ad, np, n, A, invN / (double)n))) return rc;
+            if ((rc = fac_gram(f, bd, mp, m, B))) return rc;
         }
     }
     return KG_OK;

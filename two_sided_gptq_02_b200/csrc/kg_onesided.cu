@@ -13,24 +13,24 @@
 // sequence with the in-block updates applied at once (U_A's block broadcast from shared memory).
 // solve(J0, J1) recurses over blocks: solve [J0, mid), then
 //     W~[:, mid..J1) -= E[:, J0..mid) U_A[J0..mid, mid..J1)
-// -- one dense GEMM on the tensor cores, cuBLAS: fp32 emulated with three bf16 terms per operand
-// (BF16x9, fp32 accuracy), fp64 DGEMM -- then solve [mid, J1).  Rows never interact, so the
-// leaves need no anti-diagonal wavefront and there is no second chain.
-#include <cublas_v2.h>
-
+// -- one dense GEMM on the tensor cores: fp32 on tcgen05 with 3xTF32 (k_gemm_tc32: E and U_A^T
+// kept as split tf32 planes, staged by TMA, accumulated in TMEM), fp64 on the FP64 tensor path
+// (mma.sync m8n8k4, kg_dgemm.cuh) -- then solve [mid, J1).  Rows never interact, so the leaves
+// need no anti-diagonal wavefront and there is no second chain.  W~ and E are padded to a
+// multiple of 64 rows (zero rows, which stay zero).
 #include <algorithm>
 #include <type_traits>
 #include <vector>
 
-#include "kg_blas.cuh"
 #include "kg_common.cuh"
+#include "kg_dgemm.cuh"
 #include "kg_profile.cuh"
+#include "kg_push_tc.cuh"
 
 namespace kg {
 
 constexpr int OS_T = 64;      // block width (columns)
 constexpr int OS_ROWS = 32;   // rows per leaf CTA (one warp)
-constexpr size_t OS_BLAS_WS = 32u << 20;
 
 template <typename Real>
 struct OsSmem {
@@ -41,19 +41,22 @@ struct OsSmem {
     int8_t cs[OS_ROWS][OS_T];
 };
 
-// W~ = W padded with zero columns to Np; W must be finite
+// W~ = W padded with zero rows and columns to Mp x Np (W must be finite); E (and its lo plane in
+// fp32) zero, so that the padded rows stay zero through every update
 template <typename Real>
-__global__ void k_os_init(const Real* __restrict__ W, int64_t m, int64_t n, int64_t Np, Real* __restrict__ Wt,
-                          DevStatus* status) {
+__global__ void k_os_init(const Real* __restrict__ W, int64_t m, int64_t n, int64_t Mp, int64_t Np,
+                          Real* __restrict__ Wt, Real* __restrict__ E, Real* __restrict__ Elo, DevStatus* status) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < m * Np; p += stride) {
+    for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < Mp * Np; p += stride) {
         const int64_t i = p / Np, j = p - i * Np;
         Real v = Real(0);
-        if (j < n) {
+        if (i < m && j < n) {
             v = W[i * n + j];
             if (!isfinite(v)) set_status(status, KG_ERR_NONFINITE, (int)(i * n + j < INT32_MAX ? i * n + j : INT32_MAX));
         }
         Wt[p] = v;
+        E[p] = Real(0);
+        if (Elo) Elo[p] = Real(0);
     }
 }
 
@@ -81,7 +84,8 @@ __global__ void k_os_pad(const Real* __restrict__ U, int64_t n, int64_t Np, Real
 // One 64-column block J for 32 rows per CTA.
 template <typename Real>
 __global__ void __launch_bounds__(OS_ROWS) k_os_leaf(int J, int64_t m, int64_t n, int64_t Np, Real* __restrict__ Wt,
-                                                     Real* __restrict__ Ebuf, const Real* __restrict__ UA, int64_t ldA,
+                                                     Real* __restrict__ Ebuf, Real* __restrict__ Elo,
+                                                     const Real* __restrict__ UA, int64_t ldA,
                                                      const Real* __restrict__ sp, int qmin, int qmax,
                                                      int8_t* __restrict__ codes, Real* __restrict__ V,
                                                      Real* __restrict__ outE) {
@@ -166,7 +170,14 @@ __global__ void __launch_bounds__(OS_ROWS) k_os_leaf(int J, int64_t m, int64_t n
         for (int h = 0; h < 2; ++h) {
             const int c = lane + 32 * h;
             const int64_t col = c0 + c;
-            Ebuf[row * Np + col] = sm.st[r][c];
+            if constexpr (sizeof(Real) == 4) {
+                float hi, lo;   // the tensor-core update reads E as tf32 hi + lo planes
+                tc::split_tf32(sm.st[r][c], hi, lo);
+                Ebuf[row * Np + col] = hi;
+                Elo[row * Np + col] = lo;
+            } else {
+                Ebuf[row * Np + col] = sm.st[r][c];
+            }
             if (col < n) {
                 codes[row * n + col] = sm.cs[r][c];
                 V[row * n + col] = sm.vq[r][c];
@@ -177,8 +188,8 @@ __global__ void __launch_bounds__(OS_ROWS) k_os_leaf(int J, int64_t m, int64_t n
 }
 
 struct OsArgs {
-    int64_t m, n, Np, Nt, ldA;
-    void *Wt, *E;
+    int64_t m, n, Mp, Np, Nt, ldA;
+    void *Wt, *E, *Elo;
     const void* UA;
     const void* sp;
     int qmin, qmax;
@@ -186,7 +197,8 @@ struct OsArgs {
     void* V;
     void* outE;
     cudaStream_t st;
-    cublasHandle_t blas;
+    DevStatus* status;
+    const CUtensorMap *mEh, *mEl, *mUh, *mUl;   // fp32: E and U_A^T split planes
 };
 
 template <typename Real>
@@ -194,36 +206,30 @@ static int os_leaf(const OsArgs& a, int J) {
     ProfScope ps(PK_LEAF, a.st);
     const int grid = (int)ceil_div(a.m, OS_ROWS);
     k_os_leaf<Real><<<grid, OS_ROWS, sizeof(OsSmem<Real>), a.st>>>(
-        J, a.m, a.n, a.Np, static_cast<Real*>(a.Wt), static_cast<Real*>(a.E), static_cast<const Real*>(a.UA), a.ldA,
+        J, a.m, a.n, a.Np, static_cast<Real*>(a.Wt), static_cast<Real*>(a.E), static_cast<Real*>(a.Elo),
+        static_cast<const Real*>(a.UA), a.ldA,
         static_cast<const Real*>(a.sp), a.qmin, a.qmax, a.codes, static_cast<Real*>(a.V), static_cast<Real*>(a.outE));
     KG_LAUNCH_CHECK();
     return KG_OK;
 }
 
-// W~[:, mid..J1) -= E[:, J0..mid) U_A[J0..mid, mid..J1).  Row-major X (r x c, leading dimension L)
-// is column-major X^T, so cuBLAS computes W~^T -= U^T E^T with every operand in place.
+// W~[:, mid..J1) -= E[:, J0..mid) U_A[J0..mid, mid..J1) over all Mp rows
 template <typename Real>
 static int os_update(const OsArgs& a, int J0, int mid, int J1) {
     ProfScope ps(PK_PUSH, a.st);
-    const int M = (J1 - mid) * OS_T, N = (int)a.m, K = (mid - J0) * OS_T;
-    const Real* A = static_cast<const Real*>(a.UA) + (int64_t)J0 * OS_T * a.ldA + (int64_t)mid * OS_T;
-    const Real* B = static_cast<const Real*>(a.E) + (int64_t)J0 * OS_T;
-    Real* C = static_cast<Real*>(a.Wt) + (int64_t)mid * OS_T;
-    const Real one = 1, minus_one = -1;
-    cublasStatus_t s;
+    const int rows = (int)a.Mp, c0 = mid * OS_T, cols = (J1 - mid) * OS_T, k0 = J0 * OS_T, k1 = mid * OS_T;
     if constexpr (sizeof(Real) == 8) {
-        s = cublasDgemm(a.blas, CUBLAS_OP_N, CUBLAS_OP_N, M, N, K, &minus_one, A, (int)a.ldA, B, (int)a.Np, &one, C,
-                        (int)a.Np);
+        const double* A = static_cast<const double*>(a.E) + k0;
+        const double* B = static_cast<const double*>(a.UA) + (int64_t)k0 * a.ldA + c0;
+        double* C = static_cast<double*>(a.Wt) + c0;
+        return dgemm(a.st, 0, rows, cols, k1 - k0, -1.0, A, a.Np, B, a.ldA, 1.0, C, a.Np) ? KG_OK : KG_ERR_CUDA;
     } else {
-        s = cublasGemmEx(a.blas, CUBLAS_OP_N, CUBLAS_OP_N, M, N, K, &minus_one, A, CUDA_R_32F, (int)a.ldA, B,
-                         CUDA_R_32F, (int)a.Np, &one, C, CUDA_R_32F, (int)a.Np, CUBLAS_COMPUTE_32F_EMULATED_16BFX9,
-                         CUBLAS_GEMM_DEFAULT);
-        if (s != CUBLAS_STATUS_SUCCESS)   // plain fp32 GEMM where the emulation is not offered
-            s = cublasGemmEx(a.blas, CUBLAS_OP_N, CUBLAS_OP_N, M, N, K, &minus_one, A, CUDA_R_32F, (int)a.ldA, B,
-                             CUDA_R_32F, (int)a.Np, &one, C, CUDA_R_32F, (int)a.Np, CUBLAS_COMPUTE_32F,
-                             CUBLAS_GEMM_DEFAULT);
+        const dim3 grid((unsigned)ceil_div(cols, 128), (unsigned)ceil_div(rows, 128));
+        k_gemm_tc32<<<grid, PushCfg<2>::THREADS, PushCfg<2>::SMEM_BYTES, a.st>>>(
+            rows, c0, cols, k0, k1, static_cast<float*>(a.Wt), a.Np, *a.mEh, *a.mEl, *a.mUh, *a.mUl, a.status);
+        KG_LAUNCH_CHECK();
+        return KG_OK;
     }
-    return s == CUBLAS_STATUS_SUCCESS ? KG_OK : KG_ERR_CUDA;
 }
 
 template <typename Real>
@@ -236,22 +242,30 @@ static int os_solve(const OsArgs& a, int J0, int J1) {
     return os_solve<Real>(a, mid, J1);
 }
 
+// Workspace: [status][W~ Mp*Np][E Mp*Np][padded U_A Np*Np, when n % 64 != 0]
+//            fp32 only: [E lo plane Mp*Np][U_A^T hi Np*Np][U_A^T lo Np*Np]
 struct OsLayout {
-    int64_t Np;
-    size_t off_wt, off_e, off_ua, off_blas, total;
+    int64_t Mp, Np;
+    size_t off_wt, off_e, off_ua, off_elo, off_uath, off_uatl, total;
     bool padded;
 };
 
 static OsLayout os_layout(int64_t m, int64_t n, size_t es) {
     OsLayout L{};
+    L.Mp = ceil_div(m, OS_T) * OS_T;
     L.Np = ceil_div(n, OS_T) * OS_T;
     L.padded = L.Np != n;
     size_t off = kStatusBytes;
-    L.off_wt = off;   off = align_up(off + (size_t)(m * L.Np) * es, 256);
-    L.off_e = off;    off = align_up(off + (size_t)(m * L.Np) * es, 256);
+    L.off_wt = off;   off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
+    L.off_e = off;    off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
     L.off_ua = off;
     if (L.padded) off = align_up(off + (size_t)(L.Np * L.Np) * es, 256);
-    L.off_blas = off; off += OS_BLAS_WS;
+    L.off_elo = L.off_uath = L.off_uatl = off;
+    if (es == 4) {
+        L.off_elo = off;  off = align_up(off + (size_t)(L.Mp * L.Np) * es, 256);
+        L.off_uath = off; off = align_up(off + (size_t)(L.Np * L.Np) * es, 256);
+        L.off_uatl = off; off = align_up(off + (size_t)(L.Np * L.Np) * es, 256);
+    }
     L.total = off;
     return L;
 }
@@ -263,20 +277,20 @@ static int quantize_onesided_impl(const void* W, int64_t m, int64_t n, const voi
     unsigned char* base = static_cast<unsigned char*>(ws);
     DevStatus* status = reinterpret_cast<DevStatus*>(base);
     OsArgs a{};
-    a.m = m; a.n = n; a.Np = L.Np; a.Nt = L.Np / OS_T;
+    a.m = m; a.n = n; a.Mp = L.Mp; a.Np = L.Np; a.Nt = L.Np / OS_T;
     a.Wt = base + L.off_wt;
     a.E = base + L.off_e;
+    a.Elo = sizeof(Real) == 4 ? base + L.off_elo : nullptr;
     a.sp = grid.row_scale;
     a.qmin = grid.qmin; a.qmax = grid.qmax;
     a.codes = codes; a.V = V; a.outE = outE; a.st = st;
-    int rc = blas_handle(&a.blas);
-    if (!rc) rc = blas_bind(a.blas, st, base + L.off_blas, OS_BLAS_WS);
-    if (rc) return rc;
+    a.status = status;
     const int nb = 148 * 4;
     KG_CUDA_TRY(cudaMemsetAsync(status, 0, kStatusBytes, st));
     {
         ProfScope ps(PK_INIT, st);
-        k_os_init<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(W), m, n, L.Np, static_cast<Real*>(a.Wt), status);
+        k_os_init<Real><<<nb, 256, 0, st>>>(static_cast<const Real*>(W), m, n, L.Mp, L.Np, static_cast<Real*>(a.Wt),
+                                            static_cast<Real*>(a.E), static_cast<Real*>(a.Elo), status);
     }
     KG_LAUNCH_CHECK();
     {
@@ -295,6 +309,21 @@ static int quantize_onesided_impl(const void* W, int64_t m, int64_t n, const voi
         a.UA = UA;
         a.ldA = n;
     }
+    CUtensorMap maps[4];
+    if constexpr (sizeof(Real) == 4) {
+        float* uath = reinterpret_cast<float*>(base + L.off_uath);
+        float* uatl = reinterpret_cast<float*>(base + L.off_uatl);
+        {
+            ProfScope ps(PK_INIT, st);
+            k_transpose_split<<<nb, 256, 0, st>>>(static_cast<const float*>(a.UA), L.Np, a.ldA, uath, uatl);
+        }
+        KG_LAUNCH_CHECK();
+        if (!push_tma_map(&maps[0], static_cast<const float*>(a.E), L.Np, L.Mp) ||
+            !push_tma_map(&maps[1], static_cast<const float*>(a.Elo), L.Np, L.Mp) ||
+            !push_tma_map(&maps[2], uath, L.Np, L.Np) || !push_tma_map(&maps[3], uatl, L.Np, L.Np))
+            return KG_ERR_CUDA;
+        a.mEh = &maps[0]; a.mEl = &maps[1]; a.mUh = &maps[2]; a.mUl = &maps[3];
+    }
     return os_solve<Real>(a, 0, (int)a.Nt);
 }
 
@@ -302,6 +331,12 @@ template <typename Real>
 static int os_configure() {
     KG_CUDA_TRY(cudaFuncSetAttribute(k_os_leaf<Real>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)sizeof(OsSmem<Real>)));
+    if constexpr (sizeof(Real) == 4) {
+        KG_CUDA_TRY(cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         PushCfg<2>::SMEM_BYTES));
+        KG_CUDA_TRY(cudaFuncSetAttribute(k_gemm_tc32, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared));
+    }
     return KG_OK;
 }
 

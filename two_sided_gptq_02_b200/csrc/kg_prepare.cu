@@ -7,15 +7,20 @@
 // P A_d P = L' L'^T (ordinary lower Cholesky), hence A_d = (P L' P)(P L' P)^T with P L' P
 // upper, and U = (P L' P)^{-1} = P L'^{-1} P.  So the GPU computes
 //     1. M  = P A_d P                      (copy with reversal and damping, padded to 64)
-//     2. L' = Cholesky(M)                  (right-looking, 64x64 blocks)
-//     3. X  = L'^{-1}                      (blocked lower-triangular inverse)
-//     4. U[i][j] = X[k-1-i][k-1-j]         (reversal back; strictly lower part zero)
-// Two O(k^3) steps instead of the three of "Cholesky, inverse, Cholesky of the inverse";
-// the result is the same unique factor.  Every block product runs on the FP64 tensor path
-// (mma.sync m8n8k4 f64) through kg::Dmma64.
+//     2. L' = Cholesky(M), X = L'^{-1}     (one recursion that halves the block range: factor
+//                                           and invert the leading half, update and factor
+//                                           the trailing half, then the off-diagonal block of
+//                                           the inverse; 64 x 64 leaves in one CTA)
+//     3. U[i][j] = X[k-1-i][k-1-j]         (reversal back; strictly lower part zero)
+// The Cholesky and the triangular inverse ("FastKron", Section 2.6: inverse and Cholesky as a
+// separate O(n^3) step) instead of the three steps of "Cholesky, inverse, Cholesky of the
+// inverse"; the result is the same unique factor.  The recursion's sequential depth is the 64
+// leaves; every product between them is one DGEMM on the FP64 tensor path (mma.sync m8n8k4 f64,
+// kg_dgemm.cuh) over whole half-blocks.
 #include <algorithm>
 
 #include "kg_common.cuh"
+#include "kg_dgemm.cuh"
 #include "kg_gemm.cuh"
 #include "kg_profile.cuh"
 
@@ -25,7 +30,7 @@ constexpr int NB = 64;
 
 struct PLayout {
     int64_t k, kp, Kb;
-    size_t off_scal, off_M, off_X, off_Dinv, off_Tmp, total;
+    size_t off_scal, off_M, off_X, off_T, total;
 };
 
 static PLayout p_layout(int64_t k) {
@@ -37,8 +42,7 @@ static PLayout p_layout(int64_t k) {
     L.off_scal = off; off += 256;
     L.off_M = off;    off = align_up(off + (size_t)(L.kp * L.kp) * 8, 256);
     L.off_X = off;    off = align_up(off + (size_t)(L.kp * L.kp) * 8, 256);
-    L.off_Dinv = off; off = align_up(off + (size_t)(L.kp * NB) * 8, 256);
-    L.off_Tmp = off;  off = align_up(off + (size_t)(L.kp * NB) * 8, 256);
+    L.off_T = off;    off = align_up(off + (size_t)(L.kp * L.kp) * 8, 256);
     L.total = off;
     return L;
 }
@@ -85,138 +89,187 @@ __global__ void k_build_reversed(const In* __restrict__ A, int64_t k, int64_t kp
     }
 }
 
-// Factor the diagonal block M[kb,kb] in place (lower Cholesky) and write its inverse to
-// Dinv[kb] (64 x 64, row-major).  One block of 256 threads.
+// Leaf of the recursion: the 64 x 64 diagonal block at (o, o).  In place, its lower triangle
+// becomes the Cholesky factor L; X[o.., o..] receives L^{-1} (lower, zero above the diagonal).
+// One CTA of 256 threads, thread (ty, tx) owning the 4 x 4 block of rows 4ty.., columns 4tx.. in
+// registers.  Cholesky, right-looking by columns: the owner of the pivot takes its square root,
+// the owners of column c publish L[r][c] = a[r][c] / L[c][c], every thread subtracts
+// L[r][c] L[c'][c] from its entries (c < c' <= r).  The inverse by rows: once row t of X is final
+// (divided by L[t][t]), every row r > t subtracts L[r][t] X[t][:].  Two barriers a step.
 __global__ void __launch_bounds__(256)
-k_potrf_diag(double* __restrict__ M, int64_t kp, int kb, int64_t k, double* __restrict__ Dinv, DevStatus* st) {
-    __shared__ double Ls[NB][NB + 1];
-    const int tid = threadIdx.x;
-    double* blk = M + (int64_t)kb * NB * kp + (int64_t)kb * NB;
-    for (int idx = tid; idx < NB * NB; idx += 256) {
-        const int r = idx / NB, c = idx % NB;
-        Ls[r][c] = (c <= r) ? blk[(int64_t)r * kp + c] : 0.0;
-    }
-    __syncthreads();
+k_chol_inv64(double* __restrict__ M, double* __restrict__ X, int64_t kp, int64_t o, int64_t k, DevStatus* st) {
+    __shared__ double colv[NB];          // column c of L (Cholesky) / row t of X (inverse)
+    __shared__ double Ls[NB][NB + 1];    // L, for the inverse
+    __shared__ double piv;
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    const int r0 = 4 * ty, c0 = 4 * tx;
+    double* blk = M + o * kp + o;
+    double a[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[i][j] = (c0 + j <= r0 + i) ? blk[(int64_t)(r0 + i) * kp + c0 + j] : 0.0;
     for (int c = 0; c < NB; ++c) {
-        if (tid == 0) {
-            double pv = Ls[c][c];
+        const int cb = c >> 2, cj = c & 3;
+        if (tx == cb && ty == cb) {
+            double pv = 0.0;   // a[cj][cj], selected with static register indices
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (i == cj && j == cj) pv = a[i][j];
             if (!(pv > 0.0) || !isfinite(pv)) {
-                const int64_t orig = k - 1 - ((int64_t)kb * NB + c);
-                set_status(st, KG_ERR_NOT_PD, (int)orig);
+                set_status(st, KG_ERR_NOT_PD, (int)(k - 1 - (o + c)));
                 pv = 1.0;
             }
-            Ls[c][c] = sqrt(pv);
+            piv = sqrt(pv);
         }
         __syncthreads();
-        const double d = Ls[c][c];
-        for (int r = c + 1 + tid; r < NB; r += 256) Ls[r][c] /= d;
+        const double d = piv;
+        if (tx == cb) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                double v = 0.0;   // a[i][cj]
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j == cj) v = a[i][j];
+                const int r = r0 + i;
+                if (r >= c) {
+                    v = (r == c) ? d : v / d;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (j == cj) a[i][j] = v;
+                    colv[r] = v;
+                    Ls[r][c] = v;
+                }
+            }
+        }
         __syncthreads();
-        // trailing update of the lower triangle: Ls[r][cc] -= Ls[r][c] * Ls[cc][c], c < cc <= r
-        const int rem = NB - c - 1;
-        for (int idx = tid; idx < rem * rem; idx += 256) {
-            const int r = c + 1 + idx / rem, cc = c + 1 + idx % rem;
-            if (cc <= r) Ls[r][cc] -= Ls[r][c] * Ls[cc][c];
+        // trailing update of the lower triangle right of column c
+        if (r0 + 3 > c && c0 + 3 > c) {
+            double lr[4], lc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) lr[i] = (r0 + i > c) ? colv[r0 + i] : 0.0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) lc[j] = (c0 + j > c) ? colv[c0 + j] : 0.0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (c0 + j <= r0 + i) a[i][j] -= lr[i] * lc[j];
         }
         __syncthreads();
     }
-    for (int idx = tid; idx < NB * NB; idx += 256) {
-        const int r = idx / NB, c = idx % NB;
-        blk[(int64_t)r * kp + c] = (c <= r) ? Ls[r][c] : 0.0;
-    }
-    // inverse X = L^{-1}, row by row: X[r][c] = (delta_rc - sum_{c<=t<r} L[r][t] X[t][c]) / L[r][r].
-    // The strictly lower part of X is kept transposed in the free upper triangle of Ls
-    // (Ls[c][r] = X[r][c], c < r); the diagonals live in dg / xd.
-    __shared__ double dg[NB], xd[NB];
-    if (tid < NB) dg[tid] = Ls[tid][tid];
-    __syncthreads();
-    for (int r = 0; r < NB; ++r) {
-        for (int c = tid; c <= r; c += 256) {
-            if (c == r) {
-                xd[r] = 1.0 / dg[r];
-            } else {
-                double s = -Ls[r][c] * xd[c];
-                for (int t = c + 1; t < r; ++t) s -= Ls[r][t] * Ls[c][t];
-                Ls[c][r] = s / dg[r];
+    // L back to the block (lower triangle; the upper triangle of the block is left as it was)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (c0 + j <= r0 + i) blk[(int64_t)(r0 + i) * kp + c0 + j] = a[i][j];
+    // inverse: x starts as the identity; row t is divided by L[t][t], then removed from the rows below
+    double x[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[i][j] = (r0 + i == c0 + j) ? 1.0 : 0.0;
+    for (int t = 0; t < NB; ++t) {
+        const int tb = t >> 2, ti = t & 3;
+        if (ty == tb) {
+            const double inv = 1.0 / Ls[t][t];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i == ti) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        x[i][j] *= inv;
+                        colv[c0 + j] = x[i][j];
+                    }
+                }
+        }
+        __syncthreads();
+        if (r0 + 3 > t && c0 <= t) {
+            double xr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xr[j] = colv[c0 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = r0 + i;
+                if (r > t) {
+                    const double l = Ls[r][t];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[i][j] -= l * xr[j];
+                }
             }
         }
         __syncthreads();
     }
-    double* Di = Dinv + (int64_t)kb * NB * NB;
-    for (int idx = tid; idx < NB * NB; idx += 256) {
-        const int r = idx / NB, c = idx % NB;
-        double v = 0.0;
-        if (c == r) v = xd[r];
-        else if (c < r) v = Ls[c][r];
-        Di[(int64_t)r * NB + c] = v;
-    }
+    double* xb = X + o * kp + o;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xb[(int64_t)(r0 + i) * kp + c0 + j] = (c0 + j <= r0 + i) ? x[i][j] : 0.0;
 }
 
-// L[ib,kb] = M[ib,kb] * Dinv[kb]^T for ib = kb+1 .. Kb-1 (in place; each block owns its tile)
-__global__ void __launch_bounds__(Dmma64::kThreads)
-k_panel(double* __restrict__ M, int64_t kp, int kb, const double* __restrict__ Dinv) {
-    using Pipe = DmmaPipe<false, true>;
-    __shared__ Pipe::Smem sm;
-    const int ib = kb + 1 + blockIdx.x;
-    double* tile = M + (int64_t)ib * NB * kp + (int64_t)kb * NB;
-    Dmma64::Acc acc;
-    Dmma64::zero(acc);
-    Pipe::run(acc, sm, NB, tile, kp, Dinv + (int64_t)kb * NB * NB, NB);
-    __syncthreads();
-    Dmma64::for_each(acc, [&](int r, int c, double v) { tile[(int64_t)r * kp + c] = v; });
-}
-
-// M[ib,jb] -= L[ib,kb] L[jb,kb]^T for kb < jb <= ib
-__global__ void __launch_bounds__(Dmma64::kThreads)
-k_syrk(double* __restrict__ M, int64_t kp, int kb) {
-    using Pipe = DmmaPipe<false, true>;
-    __shared__ Pipe::Smem sm;
-    const int jb = kb + 1 + blockIdx.x;
-    const int ib = kb + 1 + blockIdx.y;
-    if (jb > ib) return;
-    Dmma64::Acc acc;
-    Dmma64::zero(acc);
-    Pipe::run(acc, sm, NB, M + (int64_t)ib * NB * kp + (int64_t)kb * NB, kp,
-              M + (int64_t)jb * NB * kp + (int64_t)kb * NB, kp);
-    Dmma64::add_to(acc, M + (int64_t)ib * NB * kp + (int64_t)jb * NB, kp, -1.0);
-}
-
-// X[ib,ib] = Dinv[ib] and zero the strictly upper block triangle of X
-__global__ void k_x_init(double* __restrict__ X, int64_t kp, const double* __restrict__ Dinv) {
-    const int64_t total = kp * kp;
+// dst[r][c] = src[r][c] on an n_r x n_c block (both leading dimension ld)
+__global__ void k_copy_block(const double* __restrict__ src, double* __restrict__ dst, int64_t ld, int64_t n_r,
+                             int64_t n_c) {
+    const int64_t total = n_r * n_c;
     for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < total; p += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = p / kp, c = p % kp;
-        const int64_t rb = r / NB, cb = c / NB;
-        double v = 0.0;
-        if (rb == cb) v = Dinv[(rb * NB + (r % NB)) * NB + (c % NB)];
-        X[p] = v;
+        const int64_t r = p / n_c, c = p % n_c;
+        dst[r * ld + c] = src[r * ld + c];
     }
 }
 
-// Tmp[:, jb] = sum_{kb=jb}^{ib-1} L[ib,kb] X[kb,jb]    for jb < ib
-__global__ void __launch_bounds__(Dmma64::kThreads)
-k_inv_accum(const double* __restrict__ M, const double* __restrict__ X, int64_t kp, int ib, double* __restrict__ Tmp) {
-    using Pipe = DmmaPipe<false, false>;
-    __shared__ Pipe::Smem sm;
-    const int jb = blockIdx.x;
-    Dmma64::Acc acc;
-    Dmma64::zero(acc);
-    Pipe::run(acc, sm, (ib - jb) * NB, M + (int64_t)ib * NB * kp + (int64_t)jb * NB, kp,
-              X + (int64_t)jb * NB * kp + (int64_t)jb * NB, kp);
-    double* out = Tmp + (int64_t)jb * NB;
-    Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] = v; });
-}
-
-// X[ib,jb] = -Dinv[ib] * Tmp[:, jb]
-__global__ void __launch_bounds__(Dmma64::kThreads)
-k_inv_apply(double* __restrict__ X, int64_t kp, int ib, const double* __restrict__ Dinv, const double* __restrict__ Tmp) {
-    using Pipe = DmmaPipe<false, false>;
-    __shared__ Pipe::Smem sm;
-    const int jb = blockIdx.x;
-    Dmma64::Acc acc;
-    Dmma64::zero(acc);
-    Pipe::run(acc, sm, NB, Dinv + (int64_t)ib * NB * NB, NB, Tmp + (int64_t)jb * NB, kp);
-    double* out = X + (int64_t)ib * NB * kp + (int64_t)jb * NB;
-    Dmma64::for_each(acc, [&](int r, int c, double v) { out[(int64_t)r * kp + c] = -v; });
+// Recursive Cholesky with inverse of the block [o, o+n) of M (lower triangle, n a multiple of 64):
+// afterwards M's lower triangle there holds L and X holds L^{-1}.  With the split n = n1 + n2,
+//     (L11, X11) = rec(A11);  L21 = A21 X11^T;  A22 -= L21 L21^T;  (L22, X22) = rec(A22);
+//     X21 = -X22 (L21 X11)
+// (X11, X22 lower triangular; L21 and then X21 live in T, the product L21 X11 in X's own block).
+// Every product is a DGEMM on the FP64 tensor path that skips the zero tiles of the triangles.
+static int chol_inv_rec(double* M, double* X, double* T, int64_t kp, int64_t o, int64_t n, int64_t k, DevStatus* st,
+                        cudaStream_t s) {
+    if (n == NB) {
+        KG_PROF(PK_PREPARE, s, k_chol_inv64<<<1, 256, 0, s>>>(M, X, kp, o, k, st));
+        KG_LAUNCH_CHECK();
+        return KG_OK;
+    }
+    const int64_t n1 = ceil_div(n / NB, 2) * NB, n2 = n - n1;
+    int rc = chol_inv_rec(M, X, T, kp, o, n1, k, st, s);
+    if (rc) return rc;
+    double* A21 = M + (o + n1) * kp + o;
+    double* A22 = M + (o + n1) * kp + o + n1;
+    double* X11 = X + o * kp + o;
+    double* X21 = X + (o + n1) * kp + o;
+    double* X22 = X + (o + n1) * kp + o + n1;
+    double* T21 = T + (o + n1) * kp + o;
+    bool ok = true;
+    {
+        ProfScope ps(PK_PREPARE, s);
+        // L21 = A21 X11^T: op(B) = X11^T is upper triangular
+        ok = ok && dgemm(s, DG_TRANS_B | DG_B_UPPER, (int)n2, (int)n1, (int)n1, 1.0, A21, kp, X11, kp, 0.0, T21, kp);
+    }
+    {
+        ProfScope ps(PK_PREPARE, s);
+        // A22 -= L21 L21^T on the lower tiles
+        ok = ok && dgemm(s, DG_TRANS_B | DG_C_LOWER, (int)n2, (int)n2, (int)n1, -1.0, T21, kp, T21, kp, 1.0, A22, kp);
+    }
+    if (!ok) return KG_ERR_CUDA;
+    rc = chol_inv_rec(M, X, T, kp, o + n1, n2, k, st, s);
+    if (rc) return rc;
+    {
+        ProfScope ps(PK_PREPARE, s);
+        // P = L21 X11 (X11 lower triangular) into X21's place
+        ok = ok && dgemm(s, DG_B_LOWER, (int)n2, (int)n1, (int)n1, 1.0, T21, kp, X11, kp, 0.0, X21, kp);
+    }
+    {
+        ProfScope ps(PK_PREPARE, s);
+        // X21 = -X22 P (X22 lower triangular) into T, then back into X
+        ok = ok && dgemm(s, DG_A_LOWER, (int)n2, (int)n1, (int)n2, -1.0, X22, kp, X21, kp, 0.0, T21, kp);
+    }
+    if (!ok) return KG_ERR_CUDA;
+    KG_PROF(PK_PREPARE, s, k_copy_block<<<148 * 4, 256, 0, s>>>(T21, X21, kp, n2, n1));
+    KG_LAUNCH_CHECK();
+    return KG_OK;
 }
 
 // U[i][j] = X[k-1-i][k-1-j] (j >= i), 0 below the diagonal; optional fp32 copy
@@ -238,34 +291,15 @@ static int prepare_one(const In* A, int64_t k, double damp, double* U, float* U3
     double* scal = reinterpret_cast<double*>(base + L.off_scal);
     double* M = reinterpret_cast<double*>(base + L.off_M);
     double* X = reinterpret_cast<double*>(base + L.off_X);
-    double* Dinv = reinterpret_cast<double*>(base + L.off_Dinv);
-    double* Tmp = reinterpret_cast<double*>(base + L.off_Tmp);
-    const int Kb = (int)L.Kb;
+    double* T = reinterpret_cast<double*>(base + L.off_T);
     const int nb = 148 * 4;
 
     KG_PROF(PK_PREPARE, st, k_diag_mean<In><<<1, 256, 0, st>>>(A, k, scal, status));
     KG_LAUNCH_CHECK();
     KG_PROF(PK_PREPARE, st, k_build_reversed<In><<<nb, 256, 0, st>>>(A, k, L.kp, scal, damp, M, status));
     KG_LAUNCH_CHECK();
-    for (int kb = 0; kb < Kb; ++kb) {
-        KG_PROF(PK_PREPARE, st, k_potrf_diag<<<1, 256, 0, st>>>(M, L.kp, kb, k, Dinv, status));
-        KG_LAUNCH_CHECK();
-        const int rest = Kb - kb - 1;
-        if (rest > 0) {
-            KG_PROF(PK_PREPARE, st, k_panel<<<rest, Dmma64::kThreads, 0, st>>>(M, L.kp, kb, Dinv));
-            KG_LAUNCH_CHECK();
-            KG_PROF(PK_PREPARE, st, k_syrk<<<dim3(rest, rest), Dmma64::kThreads, 0, st>>>(M, L.kp, kb));
-            KG_LAUNCH_CHECK();
-        }
-    }
-    KG_PROF(PK_PREPARE, st, k_x_init<<<nb, 256, 0, st>>>(X, L.kp, Dinv));
-    KG_LAUNCH_CHECK();
-    for (int ib = 1; ib < Kb; ++ib) {
-        KG_PROF(PK_PREPARE, st, k_inv_accum<<<ib, Dmma64::kThreads, 0, st>>>(M, X, L.kp, ib, Tmp));
-        KG_LAUNCH_CHECK();
-        KG_PROF(PK_PREPARE, st, k_inv_apply<<<ib, Dmma64::kThreads, 0, st>>>(X, L.kp, ib, Dinv, Tmp));
-        KG_LAUNCH_CHECK();
-    }
+    const int rc = chol_inv_rec(M, X, T, L.kp, 0, L.kp, k, status, st);
+    if (rc) return rc;
     KG_PROF(PK_PREPARE, st, k_output<<<nb, 256, 0, st>>>(X, k, L.kp, U, U32));
     KG_LAUNCH_CHECK();
     return KG_OK;

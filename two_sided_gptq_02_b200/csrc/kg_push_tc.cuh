@@ -280,6 +280,158 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     if (warp == 0) tc::tmem_dealloc(tbase, PushTc::TMEM_COLS);
 }
 
+// ---------------------------------------------------------------------------------------
+// Rectangular form of the same engine, for the one-sided solve's batched update
+// ("FastKron", Section 2.4, GPTQ-recursive):  C[r, c] -= sum_k A(r, k) B(k, c)  over
+// rows [0, rows) (a multiple of 64) and columns [c0, c0 + cols) of C (multiples of 64), K over
+// [k0, k1) (multiples of 64), with A and B^T given as K-major split tf32 planes:
+//     A(r, k)  = mA[r][k]          (e.g. E, rows x K)
+//     B(k, c)  = mB[c][k]          (e.g. U_A^T, so B = U_A)
+// One CTA takes a 128 x 128 block (two 64-row boxes of A, two of B); boxes past the end of a map
+// read zeros, and rows or columns past the block's range are not stored.  Staging, the MMA
+// sequence, the bounded waits and the drain are those of k_push_tc32<2>.
+static __global__ void __launch_bounds__(PushCfg<2>::THREADS, 1)
+k_gemm_tc32(int rows, int c0, int cols, int k0, int k1, float* __restrict__ C, int64_t ldc,
+            const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
+            const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl, DevStatus* status) {
+    using Cfg = PushCfg<2>;
+    constexpr int S = Cfg::STAGES;
+    extern __shared__ __align__(16) unsigned char smem_tc_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_tc_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE_BYTES);
+    uint64_t* empty = full + S;
+    uint64_t* done = empty + S;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+    int* issued_s = reinterpret_cast<int*>(tslot + 1);
+    int* consumed_s = issued_s + 1;
+
+    const int r0 = 128 * blockIdx.y, cb = c0 + 128 * blockIdx.x;
+    if (r0 >= rows || cb >= c0 + cols || k0 >= k1) return;
+    const int nchunks = (k1 - k0) / Cfg::BK;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(done, 1);
+        *issued_s = 0;
+        *consumed_s = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tslot, Cfg::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tslot;
+    const bool failed = *reinterpret_cast<const volatile int*>(&status->code) != 0;
+    const int nch = failed ? 0 : nchunks;
+    bool ok = true;
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer: A rows r0, r0 + 64 and B rows (= C columns) cb, cb + 64 of each chunk
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % S;
+            if (c >= S && !tc::mbar_wait(&empty[s], (uint32_t)(((c / S) - 1) & 1), Cfg::MAX_WAIT_CYCLES, &status->code)) {
+                ok = false;
+                break;
+            }
+            unsigned char* st = smem + s * Cfg::STAGE_BYTES;
+            const int kx = k0 + c * Cfg::BK;
+            tc::mbar_arrive_expect_tx(&full[s], Cfg::CHUNK_BYTES);
+            tc::tma_load_2d(st, &mAh, kx, r0, &full[s]);
+            tc::tma_load_2d(st + Cfg::BOX_BYTES, &mAh, kx, r0 + 64, &full[s]);
+            tc::tma_load_2d(st + Cfg::A_BYTES, &mAl, kx, r0, &full[s]);
+            tc::tma_load_2d(st + Cfg::A_BYTES + Cfg::BOX_BYTES, &mAl, kx, r0 + 64, &full[s]);
+            unsigned char* sb = st + 2 * Cfg::A_BYTES;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                tc::tma_load_2d(sb + u * Cfg::BOX_BYTES, &mBh, kx, cb + 64 * u, &full[s]);
+                tc::tma_load_2d(sb + Cfg::B_BYTES + u * Cfg::BOX_BYTES, &mBl, kx, cb + 64 * u, &full[s]);
+            }
+            *reinterpret_cast<volatile int*>(issued_s) = c + 1;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer
+        const uint32_t idesc = tc::idesc_tf32(Cfg::M, Cfg::N, false, false);
+        for (int c = 0; c < nch; ++c) {
+            const int s = c % S;
+            if (!tc::mbar_wait(&full[s], (uint32_t)((c / S) & 1), Cfg::MAX_WAIT_CYCLES, &status->code)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            unsigned char* st = smem + s * Cfg::STAGE_BYTES;
+            const uint32_t sa_hi = tc::smem_u32(st), sa_lo = sa_hi + Cfg::A_BYTES;
+            const uint32_t sb_hi = sa_hi + 2 * Cfg::A_BYTES, sb_lo = sb_hi + Cfg::B_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < Cfg::BK / 8; ++ks) {
+                const uint64_t ah = tc::smem_desc_sw128(sa_hi + 32 * ks, Cfg::SBO);
+                const uint64_t al = tc::smem_desc_sw128(sa_lo + 32 * ks, Cfg::SBO);
+                const uint64_t bh = tc::smem_desc_sw128(sb_hi + 32 * ks, Cfg::SBO);
+                const uint64_t bl = tc::smem_desc_sw128(sb_lo + 32 * ks, Cfg::SBO);
+                const uint32_t acc0 = (c > 0 || ks > 0) ? 1u : 0u;
+                tc::mma_tf32(tbase, al, bh, idesc, acc0);
+                tc::mma_tf32(tbase, ah, bl, idesc, 1u);
+                tc::mma_tf32(tbase, ah, bh, idesc, 1u);
+            }
+            tc::mma_commit(&empty[s]);
+            *reinterpret_cast<volatile int*>(consumed_s) = c + 1;
+        }
+        tc::mma_commit(done);
+    }
+    if (!ok) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
+    __syncthreads();
+    const int never = 0;
+    bool drained = tc::mbar_wait(done, 0u, Cfg::MAX_WAIT_CYCLES, &never);
+    if (warp == 0 && lane == 0) {
+        const int consumed = *reinterpret_cast<volatile int*>(consumed_s);
+        const int issued = *reinterpret_cast<volatile int*>(issued_s);
+        for (int c = consumed; c < issued; ++c)
+            drained &= tc::mbar_wait(&full[c % S], (uint32_t)((c / S) & 1), Cfg::MAX_WAIT_CYCLES, &never);
+    }
+    const bool all_done = __syncthreads_and(drained) && *reinterpret_cast<volatile int*>(consumed_s) == nch;
+    if (!all_done && tid == 0) set_status(status, KG_ERR_TIMEOUT, (int)blockIdx.x);
+    tc::fence_after_sync();
+    if (all_done && !failed) {
+        // thread mrow owns row r0 + mrow; each 64-column half comes out of TMEM, then its 64 values
+        // are read, reduced and stored in one memory round trip
+        const int mrow = warp * 32 + lane;
+        const int r = r0 + mrow;
+        const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float v[64];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                tc::tmem_ld16(trow + 64 * h + q * 16, *reinterpret_cast<float(*)[16]>(&v[q * 16]));
+            tc::tmem_wait_ld();
+            const int cc = cb + 64 * h;
+            if (r >= rows || cc >= c0 + cols) continue;
+            float4* out = reinterpret_cast<float4*>(C + (int64_t)r * ldc + cc);
+            float4 o[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) o[q] = out[q];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                o[q].x -= v[4 * q + 0];
+                o[q].y -= v[4 * q + 1];
+                o[q].z -= v[4 * q + 2];
+                o[q].w -= v[4 * q + 3];
+                out[q] = o[q];
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, Cfg::TMEM_COLS);
+}
+
 // ---- host: tensor maps.  cuTensorMapEncodeTiled is a driver entry point; it is looked up once
 // through the runtime so the library needs no link-time dependency on libcuda.
 static PFN_cuTensorMapEncodeTiled_v12000 push_tma_encoder() {
@@ -319,7 +471,7 @@ static bool push_tma_maps(PushTmaMaps* mp, const SplitOperands& op, int64_t Np, 
 }
 
 // U^T split into tf32 planes: UT_hi[c][r] + UT_lo[c][r] = U[r][c] (k x k, k multiple of 32)
-__global__ void k_transpose_split(const float* __restrict__ U, int64_t k, int64_t ld, float* __restrict__ UT_hi,
+static __global__ void k_transpose_split(const float* __restrict__ U, int64_t k, int64_t ld, float* __restrict__ UT_hi,
                                   float* __restrict__ UT_lo) {
     __shared__ float t[32][33];
     const int64_t tiles = k / 32;
