@@ -98,7 +98,7 @@ KG_API const char* kron_gptq_status_string(int status);
  *     U_A = upper-triangular factor with U_A^T U_A = A_d^{-1}
  *   U_A equals RevCholesky(A_d)^{-T}; its transpose is the lower Cholesky factor of
  *   A_d^{-1} that the error feedback of "FastKron" Sec. 2.4 uses.  Computed in fp64 by a
- *   reversed blocked Cholesky of A_d and a blocked triangular inverse.
+ *   recursion that computes the reversed Cholesky factor of A_d and its inverse together.
  * Arguments:
  *   A, B      device, symmetric positive (semi)definite, row-major; dtype fac_dtype
  *             (KG_F32 is promoted to fp64).  The full matrix is read; only its lower
@@ -107,8 +107,12 @@ KG_API const char* kron_gptq_status_string(int status);
  *   damp      relative damping (>= 0); pass 0 if A, B are already damped.
  *   U_A, U_B  device outputs, fp64, n x n and m x m; the strictly lower triangle is zeroed.
  *   U_A32, U_B32  optional fp32 copies of the same factors (NULL to skip).
- *   ws        device workspace of kron_gptq_prepare_workspace_size(max(n, m)) bytes,
- *             256-byte aligned.
+ *   ws        device workspace, 256-byte aligned, of at least
+ *             kron_gptq_prepare_workspace_size(max(n, m)) bytes.  With
+ *             kron_gptq_prepare_workspace_size(n) + kron_gptq_prepare_workspace_size(m) bytes or
+ *             more, B's factor is prepared on an internal side stream (one per host thread and
+ *             device, created on first use and kept until exit) at the same time as A's; the call
+ *             still forks from and joins back into `stream`.
  * Device errors: KG_ERR_NOT_PD when a pivot of A_d or B_d is not positive (the outputs are
  *   then unspecified), KG_ERR_NONFINITE for NaN/Inf input.
  * --------------------------------------------------------------------------------------- */

@@ -224,7 +224,9 @@ def kron_gptq_prepare(A: torch.Tensor, B: torch.Tensor | None, damp: float, *, f
     UB = torch.empty(m, m, dtype=torch.float64, device=dev) if B is not None else None
     UA32 = torch.empty(n, n, dtype=torch.float32, device=dev) if fp32_copies else None
     UB32 = torch.empty(m, m, dtype=torch.float32, device=dev) if (fp32_copies and B is not None) else None
-    ws = _workspace(L.kron_gptq_prepare_workspace_size(max(n, m)), dev)
+    # a region per factor: the library then prepares the two factors side by side
+    ws_bytes = L.kron_gptq_prepare_workspace_size(n) + (L.kron_gptq_prepare_workspace_size(m) if B is not None else 0)
+    ws = _workspace(ws_bytes, dev)
     rc = L.kron_gptq_prepare(_ptr(A), n, _ptr(B), m, _dtype_code(A), float(damp), _ptr(UA), _ptr(UB),
                              _ptr(UA32), _ptr(UB32), _ptr(ws), ws.numel(), _stream(stream))
     _raise(rc, "kron_gptq_prepare")

@@ -95,60 +95,61 @@ __device__ __forceinline__ void ws_ldcol(const float* p, float (&o)[5]) {
     o[4] = p[4];
 }
 
-// The rounding warp: lane l owns rows 2l (r = 0) and 2l+1 (r = 1).
+// The rounding warp: lane l owns rows 2l (r = 0) and 2l+1 (r = 1).  The inputs of step d + 1
+// (the helpers' (P, r') and the column constants) are loaded into one of two register sets while
+// step d runs on the other; the step loop is unrolled by two so that the sets swap roles without a
+// copy (a copy at the end of the step would wait for the loads it copies: measured alone, 580
+// against 280 cycles a step).
+struct WsStepIn {
+    float pre[4];      // (P, r') of rows 2l and 2l + 1
+    float col[2][5];   // column constants of each row's column
+};
+
 __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)[2], const float (&b1)[2],
                                               const float (&b2)[2], const float (&b3)[2], const float (&sr)[2],
                                               const float (&isr)[2], const float (&ib)[2], float fqmin, float fqmax) {
-    constexpr int T = KG_T;
+    constexpr int T = KG_T, NSTEP = 2 * KG_T - 1;
     const int l = threadIdx.x & 31;
-    float cpre[4], npre[4], ccol[2][5], ncol[2][5];
-    auto load_step = [&](int d, float (&pre)[4], float (&col)[2][5]) {
-        const float4 p = *reinterpret_cast<const float4*>(&sm.pre[d % WS_RING][2 * l][0]);
-        pre[0] = p.x; pre[1] = p.y; pre[2] = p.z; pre[3] = p.w;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int j = d - 2 * l - r;
-            ws_ldcol(&sm.colc[(unsigned)j < (unsigned)T ? j : 0][0], col[r]);
-        }
-    };
     bool ok = true;   // this lane's waits so far
-    auto wait_hbar = [&](int d) {
+    auto load_step = [&](int d, WsStepIn& in) {
         if (ok && !tc::mbar_wait(&sm.hbar[d % WS_RING], (uint32_t)((d / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
                                  &sm.abort_flag)) {
             ok = false;
             sm.abort_flag = 1;   // wakes the helpers and the other lanes out of their waits
         }
+        const float4 p = *reinterpret_cast<const float4*>(&sm.pre[d % WS_RING][2 * l][0]);
+        in.pre[0] = p.x; in.pre[1] = p.y; in.pre[2] = p.z; in.pre[3] = p.w;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int j = d - 2 * l - r;
+            ws_ldcol(&sm.colc[(unsigned)j < (unsigned)T ? j : 0][0], in.col[r]);
+        }
     };
-    wait_hbar(0);
-    load_step(0, cpre, ccol);
     float e1[2] = {0.f, 0.f}, e2[2] = {0.f, 0.f}, e3[2] = {0.f, 0.f};   // own E, 1..3 steps ago
     float uo1_1 = 0.f, uo1_2 = 0.f;               // shfl_up(X_odd, 1): X of row 2l-1, 1 and 2 steps ago
     float ue1_1 = 0.f, ue1_2 = 0.f, ue1_3 = 0.f;  // shfl_up(X_even, 1): X of row 2l-2, 1..3 steps ago
     float uo2_1 = 0.f, uo2_2 = 0.f, uo2_3 = 0.f;  // shfl_up(X_odd, 2): X of row 2l-3, 1..3 steps ago
     float xe_1 = 0.f;                             // own X of row 2l, 1 step ago
-    for (int d = 0; d < 2 * T - 1; ++d) {
+    auto step = [&](int d, const WsStepIn& cur, WsStepIn& nxt) {
         // prefetch the next step's inputs; the helpers are normally ahead
-        if (d + 1 < 2 * T - 1) {
-            wait_hbar(d + 1);
-            load_step(d + 1, npre, ncol);
-        }
+        if (d + 1 < NSTEP) load_step(d + 1, nxt);
         float e[2], X[2], code[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const float xm1 = r ? xe_1 : uo1_1;    // X[i-1][j]
             const float xm2 = r ? uo1_2 : ue1_2;   // X[i-2][j]
             const float xm3 = r ? ue1_3 : uo2_3;   // X[i-3][j]
-            const float P = cpre[2 * r], rh = cpre[2 * r + 1];
+            const float P = cur.pre[2 * r], rh = cur.pre[2 * r + 1];
             // terms known before this step's chain starts
-            const float rp = (rh + e3[r] * ccol[r][2]) + e2[r] * ccol[r][1];
+            const float rp = (rh + e3[r] * cur.col[r][2]) + e2[r] * cur.col[r][1];
             const float base = ((P - b3[r] * xm3) - b2[r] * xm2) - bii[r] * rp;
             // the chain: E[i][j-1] and X[i-1][j] were made at step d-1
-            const float t1 = e1[r] * ccol[r][0];
+            const float t1 = e1[r] * cur.col[r][0];
             const float x = (base - bii[r] * t1) - b1[r] * xm1;
             code[r] = leaf_clamp(rintf(x * isr[r]), fqmin, fqmax);
             const float Q = code[r] * sr[r];
-            e[r] = (x - Q) * (ib[r] * ccol[r][3]);
-            X[r] = (rp + t1) + e[r] * ccol[r][4];
+            e[r] = (x - Q) * (ib[r] * cur.col[r][3]);
+            X[r] = (rp + t1) + e[r] * cur.col[r][4];
             const int j = d - 2 * l - r;
             if ((unsigned)j >= (unsigned)T) {
                 e[r] = 0.f;
@@ -178,14 +179,15 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             e2[r] = e1[r];
             e1[r] = e[r];
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) cpre[u] = npre[u];
-#pragma unroll
-        for (int u = 0; u < 5; ++u) {
-            ccol[0][u] = ncol[0][u];
-            ccol[1][u] = ncol[1][u];
-        }
+    };
+    WsStepIn s0, s1;
+    load_step(0, s0);
+    int d = 0;
+    for (; d + 1 < NSTEP; d += 2) {
+        step(d, s0, s1);
+        step(d + 1, s1, s0);
     }
+    step(d, s0, s1);   // NSTEP is odd: the last step
     return __all_sync(0xffffffffu, ok);
 }
 

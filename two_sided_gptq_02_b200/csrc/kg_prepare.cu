@@ -18,6 +18,7 @@
 // leaves; every product between them is one DGEMM on the FP64 tensor path (mma.sync m8n8k4 f64,
 // kg_dgemm.cuh) over whole half-blocks.
 #include <algorithm>
+#include <vector>
 
 #include "kg_common.cuh"
 #include "kg_dgemm.cuh"
@@ -305,6 +306,39 @@ static int prepare_one(const In* A, int64_t k, double damp, double* U, float* U3
     return KG_OK;
 }
 
+// the first error of the side region's status word reaches the call's status word
+__global__ void k_merge_status(DevStatus* dst, const DevStatus* src) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && src->code != 0) set_status(dst, src->code, src->detail);
+}
+
+// Per host thread and device: one non-blocking side stream and two events, created on first use and
+// kept for the life of the process, on which the output-side factor is prepared while the input-side
+// one runs on the caller's stream.
+struct PrepSide {
+    int dev = -1;
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static int prep_side(PrepSide*& out) {
+    static thread_local std::vector<PrepSide> sides;
+    int dev = 0;
+    KG_CUDA_TRY(cudaGetDevice(&dev));
+    for (auto& s : sides)
+        if (s.dev == dev) {
+            out = &s;
+            return KG_OK;
+        }
+    PrepSide s;
+    s.dev = dev;
+    KG_CUDA_TRY(cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking));
+    KG_CUDA_TRY(cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming));
+    KG_CUDA_TRY(cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming));
+    sides.push_back(s);
+    out = &sides.back();
+    return KG_OK;
+}
+
 }  // namespace kg
 
 using namespace kg;
@@ -327,13 +361,33 @@ extern "C" int kron_gptq_prepare(const void* A, int64_t n, const void* B, int64_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* base = static_cast<unsigned char*>(ws);
     KG_CUDA_TRY(cudaMemsetAsync(base, 0, kStatusBytes, st));
-    int rc;
-    if (fac_dtype == KG_F64) {
-        rc = prepare_one<double>(static_cast<const double*>(A), n, damp, U_A, U_A32, base, st);
-        if (!rc && B) rc = prepare_one<double>(static_cast<const double*>(B), m, damp, U_B, U_B32, base, st);
-    } else {
-        rc = prepare_one<float>(static_cast<const float*>(A), n, damp, U_A, U_A32, base, st);
-        if (!rc && B) rc = prepare_one<float>(static_cast<const float*>(B), m, damp, U_B, U_B32, base, st);
+    auto one = [&](const void* X, int64_t k, double* U, float* U32, unsigned char* b, cudaStream_t s) {
+        return fac_dtype == KG_F64 ? prepare_one<double>(static_cast<const double*>(X), k, damp, U, U32, b, s)
+                                   : prepare_one<float>(static_cast<const float*>(X), k, damp, U, U32, b, s);
+    };
+    // Both factors at once when the workspace holds a region for each: B on a side stream that forks
+    // from and joins back into the caller's stream, so the call stays one operation on that stream.
+    const size_t side_off = align_up(p_layout(n).total, 256);
+    if (B && ws_bytes >= side_off + p_layout(m).total) {
+        PrepSide* side = nullptr;
+        int rc = prep_side(side);
+        if (rc) return rc;
+        unsigned char* bside = base + side_off;
+        KG_CUDA_TRY(cudaMemsetAsync(bside, 0, kStatusBytes, st));
+        KG_CUDA_TRY(cudaEventRecord(side->fork, st));
+        KG_CUDA_TRY(cudaStreamWaitEvent(side->st, side->fork, 0));
+        const int rc_b = one(B, m, U_B, U_B32, bside, side->st);
+        // the join is recorded even when the side stream's launches failed, so that the caller's
+        // stream never runs ahead of work already queued there
+        KG_CUDA_TRY(cudaEventRecord(side->join, side->st));
+        rc = rc_b ? rc_b : one(A, n, U_A, U_A32, base, st);
+        KG_CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0));
+        if (rc) return rc;
+        k_merge_status<<<1, 32, 0, st>>>(reinterpret_cast<DevStatus*>(base), reinterpret_cast<const DevStatus*>(bside));
+        KG_LAUNCH_CHECK();
+        return KG_OK;
     }
+    int rc = one(A, n, U_A, U_A32, base, st);
+    if (!rc && B) rc = one(B, m, U_B, U_B32, base, st);
     return rc;
 }
