@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(256)
 k_chol_inv64(double* __restrict__ M, double* __restrict__ X, int64_t kp, int64_t o, int64_t k, DevStatus* st) {
     __shared__ double colv[NB];          // column c of L (Cholesky) / row t of X (inverse)
     __shared__ double Ls[NB][NB + 1];    // L, for the inverse
-    __shared__ double piv;
+    __shared__ double rdg[NB];           // 1 / L[c][c], one division per column
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int r0 = 4 * ty, c0 = 4 * tx;
     double* blk = M + o * kp + o;
@@ -123,10 +123,12 @@ k_chol_inv64(double* __restrict__ M, double* __restrict__ X, int64_t kp, int64_t
                 set_status(st, KG_ERR_NOT_PD, (int)(k - 1 - (o + c)));
                 pv = 1.0;
             }
-            piv = sqrt(pv);
+            const double d = sqrt(pv);
+            Ls[c][c] = d;
+            rdg[c] = 1.0 / d;
         }
         __syncthreads();
-        const double d = piv;
+        const double d = Ls[c][c], rd = rdg[c];
         if (tx == cb) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -136,7 +138,7 @@ k_chol_inv64(double* __restrict__ M, double* __restrict__ X, int64_t kp, int64_t
                     if (j == cj) v = a[i][j];
                 const int r = r0 + i;
                 if (r >= c) {
-                    v = (r == c) ? d : v / d;
+                    v = (r == c) ? d : v * rd;
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         if (j == cj) a[i][j] = v;
@@ -176,7 +178,7 @@ k_chol_inv64(double* __restrict__ M, double* __restrict__ X, int64_t kp, int64_t
     for (int t = 0; t < NB; ++t) {
         const int tb = t >> 2, ti = t & 3;
         if (ty == tb) {
-            const double inv = 1.0 / Ls[t][t];
+            const double inv = rdg[t];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 if (i == ti) {
