@@ -10,26 +10,28 @@
 // and the same outputs, but the 127 steps of the sweep are split between roles:
 //   * the rounding warp (warp 16) owns rows 2l and 2l+1 in lane l.  For entry (i, j) at step d
 //     it takes the helpers' partial sums
-//         P  = w'_ij - sum_{k<=i-4} b[k][i] X[k][j],     r' = sum_{k<=j-4} E[i][k] a[k][j]
-//     and adds the six newest terms itself: X of rows i-1..i-3 in column j and E of row i in
-//     columns j-1..j-3 (made at steps d-1..d-3; X of row i-1 is the lane's own other row or one
+//         P  = w'_ij - sum_{k<=i-6} b[k][i] X[k][j],     r' = sum_{k<=j-6} E[i][k] a[k][j]
+//     and adds the ten newest terms itself: X of rows i-1..i-5 in column j and E of row i in
+//     columns j-1..j-5 (made at steps d-1..d-5; X of row i-1 is the lane's own other row or one
 //     shuffle away).  Only the terms of step d-1 are on its dependent chain.  It publishes E, X
 //     and the code of every entry to shared memory.
-//   * two groups of eight helper warps (four threads per row) alternate steps: the group of step
-//     d starts as soon as step d-4 is published, so each group has two rounding steps to deliver
-//     (P, r') into an eight-slot ring.  A helper thread reads one column of X, one column of a and
-//     one row of E in 16-byte chunks (k = 4q + 16t + u, lanes of a quad interleaved; row stride 16
-//     (mod 32) words, so no bank conflicts) and multiplies with packed fp32x2 FMAs; the row's
-//     U_B column stays in registers.  Reads of entries published concurrently meet a zero
-//     coefficient (b and a are masked to k <= i-4 and k <= j-4), so they cannot change a sum.
+//   * four groups of four helper warps (two threads per row) take the steps in turn: the group of
+//     step d starts as soon as step d-6 is published, so each group has four rounding steps to
+//     deliver (P, r') into an eight-slot ring.  A helper thread reads one column of X, one column
+//     of a and one row of E in 16-byte chunks (k = 4q + 8t + u, the row's two threads interleaved)
+//     and multiplies with packed fp32x2 FMAs; the row's U_B column stays in registers.  Reads of
+//     entries published concurrently meet a zero coefficient (b and a are masked to k <= i-6 and
+//     k <= j-6), so they cannot change a sum.
 // Hand-off goes through mbarriers, one per ring slot: arrival releases the writer's shared-memory
 // stores, a waiting warp sleeps in try_wait, every wait is bounded in time, and on expiry the CTA
 // records a time-out and skips the rest.  Each warp leaves as a whole: a helper warp takes lane
 // 0's verdict; a rounding lane whose wait gives up raises the abort flag and skips its later
 // waits, but still runs every step, so the warp's shuffles stay converged, and the warp votes
-// once, after the last step.  No slot is reused before its previous phase was seen by
-// every waiter: the rounding warp cannot finish step d+8 before both helper groups finished step
-// d+5, and a helper cannot start step d+8 before step d+4 is published.
+// once, after the last step.  No slot is reused before its previous phase was seen by every
+// waiter: the helpers of step s wait on the slot of step s-6, and the rounding warp cannot start
+// step s before they are done, long before it publishes step s+2 into that slot again; the ring
+// slot of step s is refilled (for step s+8) only after step s+2 is published, and the rounding
+// warp read step s's entry during step s-1.
 #pragma once
 
 #include "kg_common.cuh"
@@ -38,10 +40,12 @@
 
 namespace kg {
 
-constexpr int WS_AHEAD = 4;                                  // helpers run this many steps ahead
+constexpr int WS_AHEAD = 6;                                  // helpers run this many steps ahead
 constexpr int WS_RING = 8;                                   // slots of the (P, r') ring
-constexpr int WS_GROUPS = 2;                                 // helper groups, alternating steps
-constexpr int WS_HELPERS = 256 * WS_GROUPS;                  // eight warps per group
+constexpr int WS_GROUPS = 4;                                 // helper groups, taking steps in turn
+constexpr int WS_TPR = 2;                                    // helper threads per row
+constexpr int WS_GTHREADS = KG_T * WS_TPR;                   // threads per group (four warps)
+constexpr int WS_HELPERS = WS_GTHREADS * WS_GROUPS;
 constexpr int WS_THREADS = WS_HELPERS + 32;                  // + the rounding warp
 #ifndef KG_TEST_HANDOFF_FAULT
 constexpr long long WS_MAX_WAIT_CYCLES = 50000000LL;         // ~25 ms: far beyond any hand-off
@@ -64,7 +68,7 @@ struct LeafWsSmem {
     float Ws[KG_T][S];             // w'
     float Rs[KG_T][KG_T + 1];      // R tile as loaded, added to the local X at the end
                                    // (stride 65: the column walk is conflict-free)
-    float colc[KG_T][8];           // column j: a[j-1][j], a[j-2][j], a[j-3][j], 1/a[j][j], a[j][j]
+    float colc[KG_T][8];           // column j: a[j-1][j] .. a[j-5][j], 1/a[j][j], a[j][j], unused
     float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
     float s[KG_T], invs[KG_T];
     int32_t Cs[KG_T][KG_T];        // codes (int32: the unclipped alphabet needs more than 8 bits)
@@ -73,12 +77,13 @@ struct LeafWsSmem {
     int abort_flag;
 };
 
-// partial dots of one helper lane: c = sum breg * xv, r = sum ev * av over its 16 k
-__device__ __forceinline__ void ws_dots(const float (&breg)[4][4], const float4 (&xv)[4], const float4 (&av)[4],
-                                        const float4 (&ev)[4], float& c, float& r) {
+// partial dots of one helper lane: c = sum breg * xv, r = sum ev * av over its NC chunks of 4 k
+template <int NC>
+__device__ __forceinline__ void ws_dots(const float (&breg)[NC][4], const float4 (&xv)[NC], const float4 (&av)[NC],
+                                        const float4 (&ev)[NC], float& c, float& r) {
     float2 c0 = make_float2(0.f, 0.f), c1 = c0, r0 = c0, r1 = c0;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    for (int t = 0; t < NC; ++t) {
         c0 = __ffma2_rn(make_float2(breg[t][0], breg[t][1]), make_float2(xv[t].x, xv[t].y), c0);
         c1 = __ffma2_rn(make_float2(breg[t][2], breg[t][3]), make_float2(xv[t].z, xv[t].w), c1);
         r0 = __ffma2_rn(make_float2(ev[t].x, ev[t].y), make_float2(av[t].x, av[t].y), r0);
@@ -88,26 +93,32 @@ __device__ __forceinline__ void ws_dots(const float (&breg)[4][4], const float4 
     r = (r0.x + r0.y) + (r1.x + r1.y);
 }
 
-// column constants of j: a1, a2, a3, 1/ajj, ajj
-__device__ __forceinline__ void ws_ldcol(const float* p, float (&o)[5]) {
+// column constants of j: a1 .. a5, 1/ajj, ajj (and one unused word)
+__device__ __forceinline__ void ws_ldcol(const float* p, float (&o)[8]) {
     const float4 t = *reinterpret_cast<const float4*>(p);
+    const float4 u = *reinterpret_cast<const float4*>(p + 4);
     o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
-    o[4] = p[4];
+    o[4] = u.x; o[5] = u.y; o[6] = u.z; o[7] = u.w;
 }
 
 // The rounding warp: lane l owns rows 2l (r = 0) and 2l+1 (r = 1).  The inputs of step d + 1
 // (the helpers' (P, r') and the column constants) are loaded into one of two register sets while
 // step d runs on the other; the step loop is unrolled by two so that the sets swap roles without a
-// copy (a copy at the end of the step would wait for the loads it copies: measured alone, 580
-// against 280 cycles a step).
+// copy (a copy at the end of the step would wait for the loads it copies).
 struct WsStepIn {
     float pre[4];      // (P, r') of rows 2l and 2l + 1
-    float col[2][5];   // column constants of each row's column
+    float col[2][8];   // column constants of each row's column
 };
 
-__device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)[2], const float (&b1)[2],
-                                              const float (&b2)[2], const float (&b3)[2], const float (&sr)[2],
-                                              const float (&isr)[2], const float (&ib)[2], float fqmin, float fqmax) {
+// The helpers leave out the WS_AHEAD - 1 = 5 newest terms of each chain; the rounding warp adds
+// them: E of its row in columns j-1 .. j-5 (its own, 1..5 steps old) and X of rows i-1 .. i-5 in
+// column j.  Row i - k (k >= 1) of column j was made k steps ago by lane l - o, o = ceil((k - r)/2),
+// as that lane's row of parity (r - k) & 1 (for r = 1, k = 1: the lane's own even row).  Each step
+// the lane takes, by shuffle, the new X of lane l-1 (both rows), l-2 (both) and l-3 (odd row) and
+// keeps them as long as they are needed: H<o><p>[t] is the X of row 2(l-o)+p made t steps ago.
+__device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)[2], const float (&bk)[2][6],
+                                              const float (&sr)[2], const float (&isr)[2], const float (&ib)[2],
+                                              float fqmin, float fqmax) {
     constexpr int T = KG_T, NSTEP = 2 * KG_T - 1;
     const int l = threadIdx.x & 31;
     bool ok = true;   // this lane's waits so far
@@ -125,40 +136,51 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             ws_ldcol(&sm.colc[(unsigned)j < (unsigned)T ? j : 0][0], in.col[r]);
         }
     };
-    float e1[2] = {0.f, 0.f}, e2[2] = {0.f, 0.f}, e3[2] = {0.f, 0.f};   // own E, 1..3 steps ago
-    float uo1_1 = 0.f, uo1_2 = 0.f;               // shfl_up(X_odd, 1): X of row 2l-1, 1 and 2 steps ago
-    float ue1_1 = 0.f, ue1_2 = 0.f, ue1_3 = 0.f;  // shfl_up(X_even, 1): X of row 2l-2, 1..3 steps ago
-    float uo2_1 = 0.f, uo2_2 = 0.f, uo2_3 = 0.f;  // shfl_up(X_odd, 2): X of row 2l-3, 1..3 steps ago
-    float xe_1 = 0.f;                             // own X of row 2l, 1 step ago
+    float eh[2][6];   // eh[r][k]: own E of row r, k steps ago (k = 1..5)
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int k = 0; k < 6; ++k) eh[r][k] = 0.f;
+    float H11[3] = {0.f, 0.f, 0.f}, H10[4] = {0.f, 0.f, 0.f, 0.f};
+    float H21[5] = {0.f, 0.f, 0.f, 0.f, 0.f}, H20[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float H31[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float xe_1 = 0.f;   // own X of row 2l, 1 step ago
     auto step = [&](int d, const WsStepIn& cur, WsStepIn& nxt) {
         // prefetch the next step's inputs; the helpers are normally ahead
         if (d + 1 < NSTEP) load_step(d + 1, nxt);
         float e[2], X[2], code[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            const float xm1 = r ? xe_1 : uo1_1;    // X[i-1][j]
-            const float xm2 = r ? uo1_2 : ue1_2;   // X[i-2][j]
-            const float xm3 = r ? ue1_3 : uo2_3;   // X[i-3][j]
+            // X[i-k][j], k = 1..5
+            const float xm1 = r ? xe_1 : H11[1];
+            const float xm2 = r ? H11[2] : H10[2];
+            const float xm3 = r ? H10[3] : H21[3];
+            const float xm4 = r ? H21[4] : H20[4];
+            const float xm5 = r ? H20[5] : H31[5];
+            const float* a = cur.col[r];
             const float P = cur.pre[2 * r], rh = cur.pre[2 * r + 1];
             // terms known before this step's chain starts
-            const float rp = (rh + e3[r] * cur.col[r][2]) + e2[r] * cur.col[r][1];
-            const float base = ((P - b3[r] * xm3) - b2[r] * xm2) - bii[r] * rp;
+            const float rp = (((rh + eh[r][5] * a[4]) + eh[r][4] * a[3]) + eh[r][3] * a[2]) + eh[r][2] * a[1];
+            const float base =
+                ((((P - bk[r][5] * xm5) - bk[r][4] * xm4) - bk[r][3] * xm3) - bk[r][2] * xm2) - bii[r] * rp;
             // the chain: E[i][j-1] and X[i-1][j] were made at step d-1
-            const float t1 = e1[r] * cur.col[r][0];
-            const float x = (base - bii[r] * t1) - b1[r] * xm1;
+            const float t1 = eh[r][1] * a[0];
+            const float x = (base - bii[r] * t1) - bk[r][1] * xm1;
             code[r] = leaf_clamp(rintf(x * isr[r]), fqmin, fqmax);
             const float Q = code[r] * sr[r];
-            e[r] = (x - Q) * (ib[r] * cur.col[r][3]);
-            X[r] = (rp + t1) + e[r] * cur.col[r][4];
+            e[r] = (x - Q) * (ib[r] * a[5]);
+            X[r] = (rp + t1) + e[r] * a[6];
             const int j = d - 2 * l - r;
             if ((unsigned)j >= (unsigned)T) {
                 e[r] = 0.f;
                 X[r] = 0.f;
             }
         }
-        const float u_o1 = __shfl_up_sync(0xffffffffu, X[1], 1);
-        const float u_e1 = __shfl_up_sync(0xffffffffu, X[0], 1);
-        const float u_o2 = __shfl_up_sync(0xffffffffu, X[1], 2);
+        const float n11 = __shfl_up_sync(0xffffffffu, X[1], 1);
+        const float n10 = __shfl_up_sync(0xffffffffu, X[0], 1);
+        const float n21 = __shfl_up_sync(0xffffffffu, X[1], 2);
+        const float n20 = __shfl_up_sync(0xffffffffu, X[0], 2);
+        const float n31 = __shfl_up_sync(0xffffffffu, X[1], 3);
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int i = 2 * l + r, j = d - i;
@@ -169,15 +191,27 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
             }
         }
         tc::mbar_arrive(&sm.cbar[d % WS_RING]);
-        uo1_2 = uo1_1; uo1_1 = u_o1;
-        ue1_3 = ue1_2; ue1_2 = ue1_1; ue1_1 = u_e1;
-        uo2_3 = uo2_2; uo2_2 = uo2_1; uo2_1 = u_o2;
+#pragma unroll
+        for (int t = 2; t > 1; --t) H11[t] = H11[t - 1];
+        H11[1] = n11;
+#pragma unroll
+        for (int t = 3; t > 1; --t) H10[t] = H10[t - 1];
+        H10[1] = n10;
+#pragma unroll
+        for (int t = 4; t > 1; --t) H21[t] = H21[t - 1];
+        H21[1] = n21;
+#pragma unroll
+        for (int t = 5; t > 1; --t) H20[t] = H20[t - 1];
+        H20[1] = n20;
+#pragma unroll
+        for (int t = 5; t > 1; --t) H31[t] = H31[t - 1];
+        H31[1] = n31;
         xe_1 = X[0];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            e3[r] = e2[r];
-            e2[r] = e1[r];
-            e1[r] = e[r];
+#pragma unroll
+            for (int k = 5; k > 1; --k) eh[r][k] = eh[r][k - 1];
+            eh[r][1] = e[r];
         }
     };
     WsStepIn s0, s1;
@@ -199,7 +233,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
           float* __restrict__ V, float* __restrict__ outE, DevStatus* status) {
     constexpr int T = KG_T;
     constexpr int VW = 4;
-    constexpr int NC = T / (4 * VW);   // chunks per lane and dot product
+    constexpr int NC = T / (WS_TPR * VW);   // chunks per lane and dot product
     constexpr int A = WS_AHEAD;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     LeafWsSmem& sm = *reinterpret_cast<LeafWsSmem*>(smem_raw);
@@ -216,8 +250,8 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     //      Es, R into XT, W~ into Ws
     if (tid == 0) {
         sm.abort_flag = 0;
-        for (int c = 0; c < 3; ++c)
-            for (int k = c; k < 3; ++k) sm.colc[c][k] = 0.f;   // a[j-k-1][j] with j-k-1 < 0
+        for (int c = 0; c < WS_AHEAD - 1; ++c)
+            for (int k = c; k < WS_AHEAD - 1; ++k) sm.colc[c][k] = 0.f;   // a[j-k-1][j] with j-k-1 < 0
     }
     if (helper) {
         // the four tiles in one memory round trip: 512 threads x 8 float4, two of each tile
@@ -243,14 +277,10 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                 if (tile == 0) {          // a: transposed, masked to k <= j-4; column constants
                     sm.aT[c][r] = (r <= c - A) ? x[u] : 0.f;
                     if (r == c) {
-                        sm.colc[c][4] = x[u];
-                        sm.colc[c][3] = 1.f / x[u];
-                    } else if (r == c - 1) {
-                        sm.colc[c][0] = x[u];
-                    } else if (r == c - 2) {
-                        sm.colc[c][1] = x[u];
-                    } else if (r == c - 3) {
-                        sm.colc[c][2] = x[u];
+                        sm.colc[c][6] = x[u];
+                        sm.colc[c][5] = 1.f / x[u];
+                    } else if (r < c && r >= c - (WS_AHEAD - 1)) {
+                        sm.colc[c][c - 1 - r] = x[u];   // a[c-k-1][c] at k = c - 1 - r
                     }
                 } else if (tile == 1) {   // b row-major, masked to the upper triangle
                     sm.Es[r][c] = (c >= r) ? x[u] : 0.f;
@@ -279,26 +309,26 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 
     // ---- per-row constants.  Helpers: U_B column of the row for k <= i-4 in registers.
     //      Rounding warp: b_ii, b[i-1][i], b[i-2][i], b[i-3][i], s_i for its two rows.
-    const int ht = tid & 255, g = tid >> 8;
-    const int i = ht >> 2, q = ht & 3;
+    const int ht = tid % WS_GTHREADS, g = tid / WS_GTHREADS;
+    const int i = ht / WS_TPR, q = ht % WS_TPR;
     float breg[NC][VW];
 #pragma unroll
     for (int t = 0; t < NC; ++t)
 #pragma unroll
         for (int u = 0; u < VW; ++u) {
-            const int k = VW * q + 4 * VW * t + u;
+            const int k = VW * q + WS_TPR * VW * t + u;
             breg[t][u] = (helper && k <= i - A) ? sm.Es[k][i] : 0.f;
         }
-    float bii[2], b1[2], b2[2], b3[2], sr[2], isr[2], ib[2];
+    float bii[2], bk[2][6], sr[2], isr[2], ib[2];
     if (!helper) {
         const int l = tid & 31;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int ir = 2 * l + r;
             bii[r] = sm.Es[ir][ir];
-            b1[r] = (ir >= 1) ? sm.Es[ir - 1][ir] : 0.f;
-            b2[r] = (ir >= 2) ? sm.Es[ir - 2][ir] : 0.f;
-            b3[r] = (ir >= 3) ? sm.Es[ir - 3][ir] : 0.f;
+            bk[r][0] = 0.f;
+#pragma unroll
+            for (int k = 1; k < 6; ++k) bk[r][k] = (ir >= k) ? sm.Es[ir - k][ir] : 0.f;
             sr[r] = sm.s[ir];
             isr[r] = sm.invs[ir];
             ib[r] = 1.f / bii[r];
@@ -343,7 +373,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     const float fqmin = (float)qmin, fqmax = (float)qmax;
     bool ok = true;
     if (!helper) {
-        ok = ws_round_warp(sm, bii, b1, b2, b3, sr, isr, ib, fqmin, fqmax);
+        ok = ws_round_warp(sm, bii, bk, sr, isr, ib, fqmin, fqmax);
     } else {
         for (int d = g; d < 2 * T - 1; d += WS_GROUPS) {
             if (d >= A) {
@@ -366,7 +396,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             float4 xv[NC], av[NC], ev[NC];
 #pragma unroll
             for (int t = 0; t < NC; ++t) {
-                const int k0 = VW * q + 4 * VW * t;
+                const int k0 = VW * q + WS_TPR * VW * t;
                 const bool pc = active && k0 <= i - A;
                 const bool pr = active && k0 <= j - A;
                 xv[t] = pc ? *reinterpret_cast<const float4*>(&sm.XT[jr][k0]) : float4{};
@@ -376,10 +406,11 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             const float w = active ? sm.Ws[i][jr] : 0.f;
             float c, r;
             ws_dots(breg, xv, av, ev, c, r);
-            c += __shfl_xor_sync(0xffffffffu, c, 1);
-            r += __shfl_xor_sync(0xffffffffu, r, 1);
-            c += __shfl_xor_sync(0xffffffffu, c, 2);
-            r += __shfl_xor_sync(0xffffffffu, r, 2);
+#pragma unroll
+            for (int o = 1; o < WS_TPR; o <<= 1) {
+                c += __shfl_xor_sync(0xffffffffu, c, o);
+                r += __shfl_xor_sync(0xffffffffu, r, o);
+            }
             if (active && q == 0) {
                 sm.pre[d % WS_RING][i][0] = w - c;
                 sm.pre[d % WS_RING][i][1] = r;
