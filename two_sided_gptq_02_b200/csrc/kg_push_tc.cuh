@@ -42,15 +42,17 @@ namespace kg {
 // NB operand tiles per CTA (N = 64 NB): NB = 2 pairs two operand tiles whose K ranges differ by
 // one tile and runs over their union; NB = 1 (small bands, where the extra tile would double the
 // work) takes one operand tile and its exact K range.
-template <int NB>
+// MT target tiles per CTA (M = 64 MT): MT = 2 for bands with several target diagonals; MT = 1 for
+// the critical part (one target diagonal: the tile next to a CTA's target never is one).
+template <int NB, int MT = 2>
 struct PushCfg {
-    static constexpr int M = 128, N = 64 * NB, BK = 32, STAGES = NB == 2 ? 3 : 4, THREADS = 128;
+    static constexpr int M = 64 * MT, N = 64 * NB, BK = 32, STAGES = NB == 2 ? 3 : 4, THREADS = 128;
     // chunk = BK = 32 K-elements = one 128-byte line per operand row
-    static constexpr int A_BYTES = M * BK * 4;                         // 16 KB per plane
+    static constexpr int A_BYTES = M * BK * 4;                         // 16 KB (MT = 2) or 8 KB per plane
     static constexpr int B_BYTES = N * BK * 4;                         // 8 KB per plane per operand tile
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;      // 64 KB (NB = 2) or 48 KB
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
     static constexpr int BOX_BYTES = 64 * BK * 4;                      // one 64-row box of one plane
-    static constexpr int CHUNK_BYTES = (4 + 2 * NB) * BOX_BYTES;       // 2 target tiles x 2 planes + B
+    static constexpr int CHUNK_BYTES = (2 * MT + 2 * NB) * BOX_BYTES;  // MT target tiles x 2 planes + B
     // + barriers (full[S], empty[S], done), TMEM slot, counters; + pad to a 1024-byte base
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
     static constexpr uint32_t TMEM_COLS = N;
@@ -92,11 +94,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 }
 }  // namespace tc
 
-template <int NB>
-__global__ void __launch_bounds__(PushCfg<NB>::THREADS, 1)
+template <int NB, int MT = 2>
+__global__ void __launch_bounds__(PushCfg<NB, MT>::THREADS, 1)
 k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float* __restrict__ Wt,
             float* __restrict__ R, const __grid_constant__ PushTmaMaps maps, DevStatus* status) {
-    using PushTc = PushCfg<NB>;
+    using PushTc = PushCfg<NB, MT>;
     constexpr int T = KG_T;
     constexpr int S = PushTc::STAGES;
     extern __shared__ __align__(16) unsigned char smem_tc_raw[];
@@ -120,7 +122,7 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     const int b0 = NB * blockIdx.x;
     if (b0 >= Bmax) return;
     const int tlo = max(0, tgt0 - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
-    const int t0 = tlo + 2 * blockIdx.y;
+    const int t0 = tlo + MT * blockIdx.y;
     if (t0 >= thi) return;
     const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
     if (k0 >= k1) return;
@@ -173,10 +175,11 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
             const int kt = k0 + c / (T / PushTc::BK);        // K tile of this chunk
             const int kx = k0 * T + c * PushTc::BK;
             tc::mbar_arrive_expect_tx(&full[s], PushTc::CHUNK_BYTES);
-            tc::tma_load_2d(st, mAh, kx, t0 * T, &full[s]);
-            tc::tma_load_2d(st + PushTc::BOX_BYTES, mAh, kx, (t0 + 1) * T, &full[s]);
-            tc::tma_load_2d(st + PushTc::A_BYTES, mAl, kx, t0 * T, &full[s]);
-            tc::tma_load_2d(st + PushTc::A_BYTES + PushTc::BOX_BYTES, mAl, kx, (t0 + 1) * T, &full[s]);
+#pragma unroll
+            for (int u = 0; u < MT; ++u) {
+                tc::tma_load_2d(st + u * PushTc::BOX_BYTES, mAh, kx, (t0 + u) * T, &full[s]);
+                tc::tma_load_2d(st + PushTc::A_BYTES + u * PushTc::BOX_BYTES, mAl, kx, (t0 + u) * T, &full[s]);
+            }
             unsigned char* sb = st + 2 * PushTc::A_BYTES;
 #pragma unroll
             for (int u = 0; u < NB; ++u) {
@@ -237,8 +240,11 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     if (all_done && !failed) {
         // Thread mrow owns accumulator row mrow (target tile t = t0 + mrow / 64).  Each 64-column
         // part (operand tile b = b0 + h) comes out of TMEM first; then all global loads of the
-        // read-modify-write are issued before any store (one memory round trip).
-        const int mrow = warp * 32 + lane;
+        // read-modify-write are issued before any store (one memory round trip).  With M = 128 row m
+        // sits in TMEM lane m; with M = 64 (MT = 1) in lane m % 16 + 32 (m / 16), so lanes 16..31
+        // of each warp hold no row.
+        const int mrow = MT == 2 ? warp * 32 + lane : warp * 16 + lane;
+        const bool row_lane = MT == 2 || lane < 16;
         const int t = t0 + (mrow >> 6), r = mrow & 63;
         const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
 #pragma unroll 1
@@ -249,7 +255,7 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
             for (int cb = 0; cb < 4; ++cb)
                 tc::tmem_ld16(trow + 64 * h + cb * 16, *reinterpret_cast<float(*)[16]>(&v[cb * 16]));
             tc::tmem_wait_ld();
-            const bool valid = t < Tmax && b < Bmax && t + b >= tgt0 && t + b < D1;
+            const bool valid = row_lane && t < Tmax && b < Bmax && t + b >= tgt0 && t + b < D1;
             if (!valid) continue;
             if (chain == 1) {
                 float4* out = reinterpret_cast<float4*>(Wt + ((int64_t)t * T + r) * Np + (int64_t)b * T);

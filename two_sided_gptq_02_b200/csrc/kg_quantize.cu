@@ -263,11 +263,16 @@ static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1,
     // in the column chain, rows of E in the row chain), y = target pair, z = chain
     ProfScope ps(PK_PUSH, st);
     // pairs of operand tiles for wide bands with several target diagonals; one target diagonal
-    // (the critical part) keeps one operand tile per CTA for twice the CTAs
+    // (the critical part) takes one operand tile and one target tile per CTA (M = 64): beside a
+    // target on that diagonal there is no second one to fill M = 128
     if (mid - D0 >= PUSH_PAIR_MIN_K && D1 - tgt0 > 1)
         return launch_k(k_push_tc32<2>, dim3((std::max(Mt, Nt) + 1) / 2, (D1 - tgt0 + 2) / 2, 2),
                         dim3(PushCfg<2>::THREADS), PushCfg<2>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt,
                         a.L.Np, a.Wt, a.R, *a.maps, a.status);
+    if (D1 - tgt0 == 1)
+        return launch_k(k_push_tc32<1, 1>, dim3(std::max(Mt, Nt), 1, 2), dim3(PushCfg<1, 1>::THREADS),
+                        PushCfg<1, 1>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps,
+                        a.status);
     return launch_k(k_push_tc32<1>, dim3(std::max(Mt, Nt), (D1 - tgt0 + 1) / 2, 2), dim3(PushCfg<1>::THREADS),
                     PushCfg<1>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps,
                     a.status);
@@ -509,6 +514,10 @@ static int configure_leaf() {
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              PushCfg<1>::SMEM_BYTES));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             PushCfg<1, 1>::SMEM_BYTES));
+            KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<1, 1>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared));
             KG_CUDA_TRY(cudaFuncSetAttribute(k_push_tc32<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              PushCfg<2>::SMEM_BYTES));
