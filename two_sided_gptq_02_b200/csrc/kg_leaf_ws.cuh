@@ -22,16 +22,21 @@
 //     and multiplies with packed fp32x2 FMAs; the row's U_B column stays in registers.  Reads of
 //     entries published concurrently meet a zero coefficient (b and a are masked to k <= i-6 and
 //     k <= j-6), so they cannot change a sum.
-// Hand-off goes through mbarriers, one per ring slot: arrival releases the writer's shared-memory
-// stores, a waiting warp sleeps in try_wait, every wait is bounded in time, and on expiry the CTA
-// records a time-out and skips the rest.  Each warp leaves as a whole: a helper warp takes lane
+// Hand-off goes through mbarriers, one phase per pair of steps (steps 2p and 2p+1): the rounding
+// warp arrives once it has published both, the helpers of both steps arrive on the pair's other
+// barrier (128 arrivals; the last, unpaired step arrives twice), so each side waits once per two
+// steps.  Arrival releases the writer's shared-memory stores, a waiting warp sleeps in try_wait,
+// every wait is bounded in time, and on expiry the CTA records a time-out and skips the rest.  Each warp leaves as a whole: a helper warp takes lane
 // 0's verdict; a rounding lane whose wait gives up raises the abort flag and skips its later
 // waits, but still runs every step, so the warp's shuffles stay converged, and the warp votes
-// once, after the last step.  No slot is reused before its previous phase was seen by every
-// waiter: the helpers of step s wait on the slot of step s-6, and the rounding warp cannot start
-// step s before they are done, long before it publishes step s+2 into that slot again; the ring
-// slot of step s is refilled (for step s+8) only after step s+2 is published, and the rounding
-// warp read step s's entry during step s-1.
+// once, after the last step.  The helpers of step s wait for the pair holding step s-6; the
+// rounding warp waits for the pair of steps 2p, 2p+1 while it runs step 2p-1, and the helpers of
+// those steps wait only for pair p-3, published after step 2p-5, so neither side waits on the other
+// in a cycle.  No barrier slot (eight pairs) is reused before its previous phase was seen by every
+// waiter: the rounding warp cannot start the steps of pair p+3 before the helpers waiting on pair p
+// are done, long before it publishes pair p+8 into that slot again; the (P, r') slot of step s is
+// refilled (for step s+8) only after step s+2 is published, and the rounding warp read it during
+// step s-1.
 #pragma once
 
 #include "kg_common.cuh"
@@ -123,8 +128,11 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
     const int l = threadIdx.x & 31;
     bool ok = true;   // this lane's waits so far
     auto load_step = [&](int d, WsStepIn& in) {
-        if (ok && !tc::mbar_wait(&sm.hbar[d % WS_RING], (uint32_t)((d / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
-                                 &sm.abort_flag)) {
+        // the helpers' sums arrive per pair of steps: wait once, before the pair's first step
+        const int pr = d >> 1;
+        if ((d & 1) == 0 && ok &&
+            !tc::mbar_wait(&sm.hbar[pr % WS_RING], (uint32_t)((pr / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
+                           &sm.abort_flag)) {
             ok = false;
             sm.abort_flag = 1;   // wakes the helpers and the other lanes out of their waits
         }
@@ -190,7 +198,7 @@ __device__ __forceinline__ bool ws_round_warp(LeafWsSmem& sm, const float (&bii)
                 sm.Cs[i][j] = (int32_t)code[r];
             }
         }
-        tc::mbar_arrive(&sm.cbar[d % WS_RING]);
+        if ((d & 1) == 1 || d == NSTEP - 1) tc::mbar_arrive(&sm.cbar[(d >> 1) % WS_RING]);
 #pragma unroll
         for (int t = 2; t > 1; --t) H11[t] = H11[t - 1];
         H11[1] = n11;
@@ -301,7 +309,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     if (tid == 0) {
         for (int k = 0; k < WS_RING; ++k) {
             tc::mbar_init(&sm.cbar[k], 32);
-            tc::mbar_init(&sm.hbar[k], T);
+            tc::mbar_init(&sm.hbar[k], 2 * T);   // both steps of a pair, one arrival per row each
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -378,7 +386,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
         for (int d = g; d < 2 * T - 1; d += WS_GROUPS) {
             if (d >= A) {
                 // step d needs everything published up to step d-4; lane 0 waits for the warp
-                const int dp = d - A;
+                const int dp = (d - A) >> 1;   // the pair holding step d - A
                 bool w_ok = true;
                 if ((tid & 31) == 0)
                     w_ok = tc::mbar_wait(&sm.cbar[dp % WS_RING], (uint32_t)((dp / WS_RING) & 1), WS_MAX_WAIT_CYCLES,
@@ -420,7 +428,11 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 #else
             constexpr bool withhold = false;
 #endif
-            if (q == 0 && !withhold) tc::mbar_arrive(&sm.hbar[d % WS_RING]);
+            if (q == 0 && !withhold) {
+                tc::mbar_arrive(&sm.hbar[(d >> 1) % WS_RING]);
+                // the last step has no partner: it completes its pair's phase alone
+                if (d == 2 * T - 2) tc::mbar_arrive(&sm.hbar[(d >> 1) % WS_RING]);
+            }
         }
     }
     if (!ok) {
