@@ -133,21 +133,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------- helpers
-def _push_flops(m, n):
+def _adjacent_pairs(Mt, Nt):
+    """(source, target) tile pairs of the near field: a tile and its right neighbour in the row
+    chain, a tile and the one below it in the column chain."""
+    return Mt * (Nt - 1) + Nt * (Mt - 1)
+
+
+def _push_flops(m, n, near_in_leaf=False):
     """FLOPs the trailing-update kernels perform per solve: each (source tile, target tile)
-    pair of the row chain and of the column chain is one 64^3 multiply-add block."""
+    pair of the row chain and of the column chain is one 64^3 multiply-add block.  With
+    near_in_leaf (the fp32 path) the adjacent pairs are the leaves' work instead."""
     Mt, Nt = math.ceil(m / TILE), math.ceil(n / TILE)
     pairs = Mt * Nt * (Nt - 1) // 2 + Nt * Mt * (Mt - 1) // 2
+    if near_in_leaf:
+        pairs -= _adjacent_pairs(Mt, Nt)
     return 2.0 * TILE ** 3 * pairs
 
 
-def _leaf_flops(m, n):
+def _leaf_flops(m, n, near_in_leaf=False):
     """FLOPs of the in-tile sweeps per solve: per 64x64 tile the two in-tile chains
     (sum over entries of j resp. i multiply-adds, 64 * 2016 each) and the fold of the external
-    row chain through the triangular U_B block (64 * 2080 multiply-adds)."""
+    row chain through the triangular U_B block (64 * 2080 multiply-adds); with near_in_leaf (the
+    fp32 leaf) also the near field, one 64^3 multiply-add block per adjacent tile pair."""
     Mt, Nt = math.ceil(m / TILE), math.ceil(n / TILE)
     per_tile = 2 * (TILE * (TILE * (TILE - 1) // 2)) + TILE * (TILE * (TILE + 1) // 2)
-    return 2.0 * per_tile * Mt * Nt
+    near = 2.0 * TILE ** 3 * _adjacent_pairs(Mt, Nt) if near_in_leaf else 0.0
+    return 2.0 * per_tile * Mt * Nt + near
 
 
 def _block_seconds(kg, torch, damp, reps=3):
@@ -672,9 +683,10 @@ def run_ours(args, rank, world, local_rank):
     ll, lms = prof["leaf"]
     il, ims = prof["init"]
     push_avg_s = pms / pl / 1e3
-    push_achieved = _push_flops(m, n) / (pl / nprof) / push_avg_s / 1e12
+    near_in_leaf = dt == torch.float32   # the fp32 leaf computes the near field itself
+    push_achieved = _push_flops(m, n, near_in_leaf) / (pl / nprof) / push_avg_s / 1e12
     leaf_avg_s = lms / ll / 1e3
-    leaf_achieved = _leaf_flops(m, n) / (ll / nprof) / leaf_avg_s / 1e12
+    leaf_achieved = _leaf_flops(m, n, near_in_leaf) / (ll / nprof) / leaf_avg_s / 1e12
     if dt == torch.float32:
         push_rl = {"bound": "tensor", "achieved": push_achieved, "peak": tf32_peak / 3.0, "unit": "TFLOP/s",
                    "frac": push_achieved / (tf32_peak / 3.0), "traffic": None, "kernel": "k_push_tc32",

@@ -31,12 +31,13 @@
  *     after them.  Errors only the device can see (a factor that is not positive definite,
  *     non-finite input, a device wait that ran out) are written to a status word inside the
  *     workspace; kron_gptq_sync_status() synchronizes the stream and returns it.
- *   - The recursive two-sided solves (quantize, quantize_noalloc, quantize_rc) run part of
- *     their update work on a second, internal stream; the caller's stream waits for it at the
- *     end, so each call stays one asynchronous operation on the caller's stream.  For this
- *     each host thread keeps, per device, eight
- *     non-blocking streams and their events (host-side driver objects, no device buffers),
- *     created on the first call and kept until the process exits.
+ *   - The recursive two-sided solves (quantize, quantize_noalloc, quantize_rc) run on four
+ *     internal streams (the leaves on one, the update pieces on the others by when they are due;
+ *     kron_gptq_schedule_plan lists them), forked from the caller's stream at the start; the
+ *     caller's stream waits for all four at the end, so each call stays one asynchronous
+ *     operation on the caller's stream.  For this each host thread keeps, per device, eight sets
+ *     of four non-blocking streams with their events (host-side driver objects, no device
+ *     buffers), created on the first call and kept until the process exits.
  *   - Concurrent calls on different streams need distinct workspaces.
  *   - Status codes: 0 = success, negative = error (see kg_status).
  */
@@ -197,9 +198,9 @@ KG_API int kron_gptq_sync_status(const void* ws, void* stream);
  *     1024 x 1024).
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current).  The first call from each host thread on a device also creates
- *     the eight internal bulk streams and their events that every recursive solve uses (host-side
- *     driver objects, no device buffers; see the conventions above).  Make both first calls
- *     before any stream capture.
+ *     the internal streams and events that every recursive solve uses (eight sets of four streams;
+ *     host-side driver objects, no device buffers; see the conventions above).  Make both first
+ *     calls before any stream capture.
  *   - All calls share the one array and each call re-initialises what it reads; calls whose
  *     executions overlap on the same GPU (different streams, threads) race on it.
  * --------------------------------------------------------------------------------------- */
@@ -349,6 +350,19 @@ KG_API int kron_gptq_quantize_antidiagonal(const void* W, int64_t m, int64_t n,
  * --------------------------------------------------------------------------------------- */
 KG_API void kron_gptq_profile_enable(int enable);
 KG_API int kron_gptq_profile_read(int64_t* launches, double* ms, int nkinds, int reset);
+
+/* ---------------------------------------------------------------------------------------
+ * kron_gptq_schedule_plan -- the update pieces kron_gptq_quantize (and _rc, _noalloc) issues for
+ *   ndiag tile anti-diagonals (ndiag = ceil(m/64) + ceil(n/64) - 1), in issue order; host only, no
+ *   device call.  The recursion of "FastKron" Section 2.5 fixes which update carries each (source,
+ *   target) pair of tile anti-diagonals; the solve cuts each update into pieces by when they are
+ *   needed.  Piece k is out[5k .. 5k+4] = {s0, s1, t0, t1, stream}: sources [s0, s1) to targets
+ *   [t0, t1); stream 0 = critical (the near piece s1 = t0 issued just before leaf t0), 1 = urgent,
+ *   2 = soon, 3 = background.  Writes at most max_pieces pieces (out may be NULL) and returns the
+ *   total count, or
+ *   KG_ERR_ARG for ndiag < 1 or max_pieces < 0.
+ * --------------------------------------------------------------------------------------- */
+KG_API int kron_gptq_schedule_plan(int ndiag, int* out, int max_pieces);
 
 #ifdef __cplusplus
 }

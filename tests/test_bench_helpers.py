@@ -31,6 +31,17 @@ def test_push_flops_approach_mn_m_plus_n():
     assert bench._push_flops(m, n) == pytest.approx(m * n * (m + n) * (1 - 64 / 4096), rel=1e-12)
 
 
+@pytest.mark.parametrize("m,n", [(64, 64), (128, 320), (1000, 130), (4096, 4096), (14336, 4096)])
+def test_near_field_moves_between_update_and_leaf(m, n):
+    # the fp32 leaf computes the adjacent-tile pairs itself: the total is conserved and the moved part
+    # is one 64^3 block per (tile, right neighbour) and (tile, lower neighbour) pair, enumerated
+    Mt, Nt = math.ceil(m / 64), math.ceil(n / 64)
+    adj = sum(1 for I in range(Mt) for J in range(1, Nt)) + sum(1 for I in range(1, Mt) for J in range(Nt))
+    moved = bench._push_flops(m, n) - bench._push_flops(m, n, near_in_leaf=True)
+    assert moved == 2.0 * 64 ** 3 * adj
+    assert bench._leaf_flops(m, n, near_in_leaf=True) - bench._leaf_flops(m, n) == moved
+
+
 def test_leaf_flops_per_tile_by_enumeration():
     T = 64
     row_chain = sum(j for i in range(T) for j in range(T))            # r_ij = sum_{k<j}

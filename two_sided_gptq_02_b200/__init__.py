@@ -19,6 +19,7 @@ Public functions mirror the C names:
     kron_gptq_factors(a, b, method, iters)          -> A, B (Kronecker factors from samples)
     kron_gptq_quantize_antidiagonal(W, U_A, U_B, ...) -> codes, V, E (quartic baseline, fp64)
     kron_gptq_sync_status(ws, stream)      -> device status word
+    kron_gptq_schedule_plan(ndiag)         -> the solve's update pieces (host only)
 """
 from __future__ import annotations
 
@@ -30,6 +31,7 @@ from ._lib import (  # noqa: F401
     RcQuantizer,
     OnesidedQuantizer,
     PROFILE_KINDS,
+    SCHEDULE_STREAMS,
     kron_gptq_loss,
     kron_gptq_profile_enable,
     kron_gptq_profile_read,
@@ -43,6 +45,7 @@ from ._lib import (  # noqa: F401
     kron_gptq_code_entropy,
     kron_gptq_waterkron_scales,
     kron_gptq_row_scales,
+    kron_gptq_schedule_plan,
     kron_gptq_status_string,
     kron_gptq_sync_status,
     kron_gptq_version,

@@ -94,6 +94,8 @@ def load_library():
         L.kron_gptq_profile_enable.restype = None
         L.kron_gptq_profile_read.argtypes = [P, P, I, I]
         L.kron_gptq_profile_read.restype = I
+        L.kron_gptq_schedule_plan.argtypes = [I, P, I]
+        L.kron_gptq_schedule_plan.restype = I
         _lib = L
         return L
 
@@ -188,6 +190,22 @@ def kron_gptq_profile_read(reset: bool = False) -> dict:
                                                  ctypes.cast(ms, ctypes.c_void_p), n, 1 if reset else 0),
            "kron_gptq_profile_read")
     return {k: (int(launches[i]), float(ms[i])) for i, k in enumerate(PROFILE_KINDS)}
+
+
+SCHEDULE_STREAMS = ("critical", "urgent", "soon", "background")
+
+
+def kron_gptq_schedule_plan(ndiag: int) -> list:
+    """The update pieces of a solve over ndiag tile anti-diagonals, in issue order:
+    [(s0, s1, t0, t1, stream)] with sources [s0, s1), targets [t0, t1) and stream an index into
+    SCHEDULE_STREAMS.  Host only."""
+    L = load_library()
+    count = L.kron_gptq_schedule_plan(int(ndiag), None, 0)
+    _raise(min(count, 0), "kron_gptq_schedule_plan")
+    buf = (ctypes.c_int * (5 * max(count, 1)))()
+    got = L.kron_gptq_schedule_plan(int(ndiag), ctypes.cast(buf, ctypes.c_void_p), count)
+    _raise(min(got, 0), "kron_gptq_schedule_plan")
+    return [tuple(buf[5 * k:5 * k + 5]) for k in range(count)]
 
 
 def kron_gptq_version() -> int:

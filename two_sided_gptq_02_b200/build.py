@@ -74,8 +74,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         f.write(flags)
     if changed:
         tmp = lib + f".{os.getpid()}.tmp"
-        # cuBLAS (the one-sided path's plain GEMM) is linked dynamically; a process that imported
-        # torch first already holds a libcublas.so.12 and the loader reuses it
+        # cuBLAS (the dense products of the anti-diagonal baseline only) is linked dynamically; a
+        # process that imported torch first already holds a libcublas.so.12 and the loader reuses it
         subprocess.check_call([NVCC, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lcublas",
                                "-Xlinker", "-rpath", "-Xlinker", CUDA_LIB])
         os.replace(tmp, lib)

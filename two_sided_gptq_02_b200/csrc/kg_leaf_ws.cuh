@@ -51,7 +51,9 @@ constexpr int WS_GROUPS = 4;                                 // helper groups, t
 constexpr int WS_TPR = 2;                                    // helper threads per row
 constexpr int WS_GTHREADS = KG_T * WS_TPR;                   // threads per group (four warps)
 constexpr int WS_HELPERS = WS_GTHREADS * WS_GROUPS;
-constexpr int WS_THREADS = WS_HELPERS + 32;                  // + the rounding warp
+constexpr int WS_PANEL = 16;                                 // columns of w' per set-up panel
+constexpr int WS_PANEL_WARPS = KG_T / WS_PANEL - 1;          // one per panel after the first
+constexpr int WS_THREADS = WS_HELPERS + 32 + 32 * WS_PANEL_WARPS;   // + the rounding warp + panel warps
 #ifndef KG_TEST_HANDOFF_FAULT
 constexpr long long WS_MAX_WAIT_CYCLES = 50000000LL;         // ~25 ms: far beyond any hand-off
 #else
@@ -71,14 +73,23 @@ struct LeafWsSmem {
     float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
     float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
     float Ws[KG_T][S];             // w'
-    float Rs[KG_T][KG_T + 1];      // R tile as loaded, added to the local X at the end
-                                   // (stride 65: the column walk is conflict-free)
     float colc[KG_T][8];           // column j: a[j-1][j] .. a[j-5][j], 1/a[j][j], a[j][j], unused
     float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
     float s[KG_T], invs[KG_T];
     int32_t Cs[KG_T][KG_T];        // codes (int32: the unclipped alphabet needs more than 8 bits)
+    // near field (set-up only): the operands of the updates from the two adjacent tiles of the
+    // previous tile anti-diagonal, each k-major ([k][row]) so that a thread reads four rows of one
+    // k in one 16-byte load
+    float Nel[KG_T][68];           // E of tile (I, J-1), transposed: [k][i] = E[i][k]
+    float Nxu[KG_T][68];           // X of tile (I-1, J): [k][j]
+    float Na[KG_T][68];            // U_A[J-1, J] block: [k][j]
+    float Nb[KG_T][68];            // U_B[I-1, I] block: [k][i]
+    float Nbd[KG_T][68];           // b = U_B[I, I] block, masked to its upper triangle: [k][i]
+    float Rp[KG_T][68];            // R of the tile with the near field added: [i][j]; the fold reads
+                                   // it, and the complete X adds it to the local X at the end
     uint64_t cbar[WS_RING];        // step d published (32 arrivals)
     uint64_t hbar[WS_RING];        // (P, r') of step d written (one arrival per row)
+    uint64_t pbar[WS_PANEL_WARPS + 1];   // w' of panel p written (32 arrivals; p >= 1)
     int abort_flag;
 };
 
@@ -243,6 +254,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     constexpr int VW = 4;
     constexpr int NC = T / (WS_TPR * VW);   // chunks per lane and dot product
     constexpr int A = WS_AHEAD;
+    constexpr int PER_ROW_Z = T / VW;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     LeafWsSmem& sm = *reinterpret_cast<LeafWsSmem*>(smem_raw);
 
@@ -251,6 +263,7 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     const int J = D - I;
     const int tid = threadIdx.x;
     const bool helper = tid < WS_HELPERS;
+    const bool rounding = !helper && tid < WS_HELPERS + 32;
     grid_dep_launch();
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
@@ -261,11 +274,24 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
         for (int c = 0; c < WS_AHEAD - 1; ++c)
             for (int k = c; k < WS_AHEAD - 1; ++k) sm.colc[c][k] = 0.f;   // a[j-k-1][j] with j-k-1 < 0
     }
+    // the adjacent tiles of the previous tile anti-diagonal: (I, J-1) sends its errors along the row
+    // chain, (I-1, J) its X down the column chain
+    const bool has_left = J > 0, has_up = I > 0;
     if (helper) {
         // the four tiles in one memory round trip: 512 threads x 8 float4, two of each tile
         const float* src[4] = {UA + c0 * ldA + c0, UB + r0 * ldB + r0, R + r0 * Np + c0, Wt + r0 * Np + c0};
         const int64_t lds[4] = {ldA, ldB, Np, Np};
-        float4 v[8];
+        // with the factor blocks of the near field: U_A[J-1, J] and U_B[I-1, I]
+        float4 v[8], nf[4];
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+            const int e = (f & 1) * WS_HELPERS + tid;
+            const bool on = f < 2 ? has_left : has_up;
+            const float* p = f < 2 ? UA + (c0 - T) * ldA + c0 : UB + (r0 - T) * ldB + r0;
+            const int64_t ld = f < 2 ? ldA : ldB;
+            nf[f] = on ? *reinterpret_cast<const float4*>(p + (int64_t)(e >> 4) * ld + (e & 15) * 4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
             // the factor tiles (f < 4) do not depend on earlier kernels of the solve: they load while
@@ -273,6 +299,43 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             if (f == 4) grid_dep_wait();
             const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;   // e: vector index in the tile
             v[f] = *reinterpret_cast<const float4*>(src[tile] + (int64_t)(e >> 4) * lds[tile] + (e & 15) * 4);
+        }
+        // the near-field sources, written by the previous leaf: E of (I, J-1) (threads 0-255) and X^T of
+        // (I-1, J) (threads 256-511), each as its two tf32 planes (hi + lo is the value to within 2^-22
+        // relative).  A thread takes a 4 x 4 block (rows 4 (q >> 4) .., columns 4 (q & 15) ..) and
+        // stores it transposed, so that both land k-major.
+        const int q = tid & 255;
+        const bool xside = tid >= 256, on = xside ? has_up : has_left;
+        const float* hi = xside ? XTg + c0 * Mp + (r0 - T) : Ebuf + r0 * Np + (c0 - T);
+        const float* lo = xside ? XTlo + c0 * Mp + (r0 - T) : Elo + r0 * Np + (c0 - T);
+        const int64_t ldn = xside ? Mp : Np;
+        float4 ns[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t off = (int64_t)(4 * (q >> 4) + u) * ldn + 4 * (q & 15);
+            ns[u] = on ? *reinterpret_cast<const float4*>(hi + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+            ns[u + 4] = on ? *reinterpret_cast<const float4*>(lo + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+            const int e = (f & 1) * WS_HELPERS + tid, r = e >> 4, c4 = (e & 15) * 4;
+            float* dst = f < 2 ? &sm.Na[r][c4] : &sm.Nb[r][c4];
+            *reinterpret_cast<float4*>(dst) = nf[f];
+        }
+        {
+            float blk[4][4];   // blk[u][w] = value at (row 4 (q >> 4) + u, column 4 (q & 15) + w)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                blk[u][0] = ns[u].x + ns[u + 4].x;
+                blk[u][1] = ns[u].y + ns[u + 4].y;
+                blk[u][2] = ns[u].z + ns[u + 4].z;
+                blk[u][3] = ns[u].w + ns[u + 4].w;
+            }
+            float(*dstT)[68] = xside ? sm.Nxu : sm.Nel;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                *reinterpret_cast<float4*>(&dstT[4 * (q & 15) + w][4 * (q >> 4)]) =
+                    make_float4(blk[0][w], blk[1][w], blk[2][w], blk[3][w]);
         }
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
@@ -291,10 +354,9 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                         sm.colc[c][c - 1 - r] = x[u];   // a[c-k-1][c] at k = c - 1 - r
                     }
                 } else if (tile == 1) {   // b row-major, masked to the upper triangle
-                    sm.Es[r][c] = (c >= r) ? x[u] : 0.f;
-                } else if (tile == 2) {   // R: for the fold (XT) and kept for the final X (Rs)
-                    sm.XT[r][c] = x[u];
-                    sm.Rs[r][c] = x[u];
+                    sm.Nbd[r][c] = (c >= r) ? x[u] : 0.f;
+                } else if (tile == 2) {   // R: the near field adds to it, the fold reads it
+                    sm.Rp[r][c] = x[u];
                 } else {
                     sm.Ws[r][c] = x[u];
                 }
@@ -305,15 +367,119 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             sm.s[tid] = s;
             sm.invs[tid] = 1.f / s;
         }
+        // Es and XT start the sweep at zero (unvisited entries contribute nothing)
+        for (int idx = tid; idx < T * T / VW; idx += WS_HELPERS) {
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(&sm.Es[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
+            *reinterpret_cast<float4*>(&sm.XT[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
+        }
     }
     if (tid == 0) {
         for (int k = 0; k < WS_RING; ++k) {
             tc::mbar_init(&sm.cbar[k], 32);
             tc::mbar_init(&sm.hbar[k], 2 * T);   // both steps of a pair, one arrival per row each
         }
+        for (int k = 1; k <= WS_PANEL_WARPS; ++k) tc::mbar_init(&sm.pbar[k], 32);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+
+    // ---- w' = W~ - U_B[I-1, I]^T X[I-1, J] - b^T R' with R' = R + E[I, J-1] U_A[J-1, J], fp32: the
+    //      near field (the updates from the adjacent tiles of tile anti-diagonal D - 1, which no update
+    //      kernel carries) and the fold of the row chain (b^T[i][k] = b[k][i] = 0 for k > i), each entry
+    //      one chain of fused multiply-adds (R' from R over k; w' from W~ over the near terms, then
+    //      over the fold terms).  In panels of 16 columns: the helpers make panel 0 before the sweep;
+    //      panel warp p - 1 makes panel p while the sweep runs, and the helpers wait for it before the
+    //      first step that reads one of its columns.
+    if (helper) {
+        const int pi = tid >> 3, pj = 2 * (tid & 7);   // row, first of two columns of panel 0
+        float2 rr = *reinterpret_cast<const float2*>(&sm.Rp[pi][pj]);
+        float2 ww = *reinterpret_cast<const float2*>(&sm.Ws[pi][pj]);
+        if (has_left) {
+#pragma unroll 8
+            for (int k = 0; k < T; ++k) {
+                const float e = sm.Nel[k][pi];
+                rr = __ffma2_rn(make_float2(e, e), *reinterpret_cast<const float2*>(&sm.Na[k][pj]), rr);
+            }
+        }
+        if (has_up) {
+#pragma unroll 8
+            for (int k = 0; k < T; ++k) {
+                const float b = -sm.Nb[k][pi];
+                ww = __ffma2_rn(make_float2(b, b), *reinterpret_cast<const float2*>(&sm.Nxu[k][pj]), ww);
+            }
+        }
+        *reinterpret_cast<float2*>(&sm.Rp[pi][pj]) = rr;
+        asm volatile("bar.sync 1, %0;" ::"n"(WS_HELPERS) : "memory");   // R' of panel 0 complete
+#pragma unroll 4
+        for (int k = 0; k <= pi; ++k) {
+            const float b = -sm.Nbd[k][pi];
+            ww = __ffma2_rn(make_float2(b, b), *reinterpret_cast<const float2*>(&sm.Rp[k][pj]), ww);
+        }
+        *reinterpret_cast<float2*>(&sm.Ws[pi][pj]) = ww;
+    } else if (!rounding) {
+        // panel warp: rows 2l, 2l + 1 of panel p
+        const int l = tid & 31, p = (tid - WS_HELPERS - 32) / 32 + 1, cb = WS_PANEL * p, ra = 2 * l;
+        float2 acc[2][WS_PANEL / 2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < WS_PANEL / 2; ++v) acc[u][v] = *reinterpret_cast<const float2*>(&sm.Rp[ra + u][cb + 2 * v]);
+        if (has_left) {
+#pragma unroll 2
+            for (int k = 0; k < T; ++k) {
+                const float2 e = *reinterpret_cast<const float2*>(&sm.Nel[k][ra]);
+#pragma unroll
+                for (int v = 0; v < WS_PANEL / 4; ++v) {
+                    const float4 x = *reinterpret_cast<const float4*>(&sm.Na[k][cb + 4 * v]);
+                    acc[0][2 * v] = __ffma2_rn(make_float2(e.x, e.x), make_float2(x.x, x.y), acc[0][2 * v]);
+                    acc[0][2 * v + 1] = __ffma2_rn(make_float2(e.x, e.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
+                    acc[1][2 * v] = __ffma2_rn(make_float2(e.y, e.y), make_float2(x.x, x.y), acc[1][2 * v]);
+                    acc[1][2 * v + 1] = __ffma2_rn(make_float2(e.y, e.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < WS_PANEL / 2; ++v) *reinterpret_cast<float2*>(&sm.Rp[ra + u][cb + 2 * v]) = acc[u][v];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < WS_PANEL / 2; ++v) acc[u][v] = *reinterpret_cast<const float2*>(&sm.Ws[ra + u][cb + 2 * v]);
+        if (has_up) {
+#pragma unroll 2
+            for (int k = 0; k < T; ++k) {
+                const float2 b = *reinterpret_cast<const float2*>(&sm.Nb[k][ra]);
+#pragma unroll
+                for (int v = 0; v < WS_PANEL / 4; ++v) {
+                    const float4 x = *reinterpret_cast<const float4*>(&sm.Nxu[k][cb + 4 * v]);
+                    acc[0][2 * v] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.x, x.y), acc[0][2 * v]);
+                    acc[0][2 * v + 1] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
+                    acc[1][2 * v] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.x, x.y), acc[1][2 * v]);
+                    acc[1][2 * v + 1] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
+                }
+            }
+        }
+        __syncwarp();   // R' of the whole panel (all rows, made by this warp) before the fold reads it
+#pragma unroll 2
+        for (int k = 0; k < T; ++k) {   // b[k][i] = 0 for k > i
+            const float2 b = *reinterpret_cast<const float2*>(&sm.Nbd[k][ra]);
+#pragma unroll
+            for (int v = 0; v < WS_PANEL / 4; ++v) {
+                const float4 x = *reinterpret_cast<const float4*>(&sm.Rp[k][cb + 4 * v]);
+                acc[0][2 * v] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.x, x.y), acc[0][2 * v]);
+                acc[0][2 * v + 1] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
+                acc[1][2 * v] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.x, x.y), acc[1][2 * v]);
+                acc[1][2 * v + 1] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int v = 0; v < WS_PANEL / 2; ++v) *reinterpret_cast<float2*>(&sm.Ws[ra + u][cb + 2 * v]) = acc[u][v];
+        tc::mbar_arrive(&sm.pbar[p]);   // every lane: its own stores are released with its arrival
+    }
 
     // ---- per-row constants.  Helpers: U_B column of the row for k <= i-4 in registers.
     //      Rounding warp: b_ii, b[i-1][i], b[i-2][i], b[i-3][i], s_i for its two rows.
@@ -325,64 +491,33 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 #pragma unroll
         for (int u = 0; u < VW; ++u) {
             const int k = VW * q + WS_TPR * VW * t + u;
-            breg[t][u] = (helper && k <= i - A) ? sm.Es[k][i] : 0.f;
+            breg[t][u] = (helper && k <= i - A) ? sm.Nbd[k][i] : 0.f;
         }
     float bii[2], bk[2][6], sr[2], isr[2], ib[2];
-    if (!helper) {
+    if (rounding) {
         const int l = tid & 31;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int ir = 2 * l + r;
-            bii[r] = sm.Es[ir][ir];
+            bii[r] = sm.Nbd[ir][ir];
             bk[r][0] = 0.f;
 #pragma unroll
-            for (int k = 1; k < 6; ++k) bk[r][k] = (ir >= k) ? sm.Es[ir - k][ir] : 0.f;
+            for (int k = 1; k < 6; ++k) bk[r][k] = (ir >= k) ? sm.Nbd[ir - k][ir] : 0.f;
             sr[r] = sm.s[ir];
             isr[r] = sm.invs[ir];
             ib[r] = 1.f / bii[r];
         }
     }
-
-    // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i);
-    //      512 threads, a 2 x 4 block each
-    {
-        const int ty = tid >> 4, tx = tid & 15;   // rows 2 ty, 2 ty + 1; columns 4 tx .. 4 tx + 3
-        float acc[2][4];
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-        if (helper) {
-            const int kmax = ty * 2 + 1;
-#pragma unroll 4
-            for (int k = 0; k <= kmax; ++k) {
-                const float2 bv = *reinterpret_cast<const float2*>(&sm.Es[k][ty * 2]);
-                const float4 rv = *reinterpret_cast<const float4*>(&sm.XT[k][tx * 4]);
-                acc[0][0] += bv.x * rv.x; acc[0][1] += bv.x * rv.y; acc[0][2] += bv.x * rv.z; acc[0][3] += bv.x * rv.w;
-                acc[1][0] += bv.y * rv.x; acc[1][1] += bv.y * rv.y; acc[1][2] += bv.y * rv.z; acc[1][3] += bv.y * rv.w;
-            }
-        }
-        __syncthreads();
-        if (helper) {
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) sm.Ws[ty * 2 + a][tx * 4 + c] -= acc[a][c];
-        }
-        // Es and XT start the sweep at zero (unvisited entries contribute nothing)
-        for (int idx = tid; idx < T * T; idx += WS_THREADS) {
-            sm.Es[idx / T][idx % T] = 0.f;
-            sm.XT[idx / T][idx % T] = 0.f;
-        }
-    }
-    __syncthreads();
+    // the helpers read w' of panel 0 made by other helpers
+    if (helper) asm volatile("bar.sync 1, %0;" ::"n"(WS_HELPERS) : "memory");
 
     // ---- sweep
     const float fqmin = (float)qmin, fqmax = (float)qmax;
     bool ok = true;
-    if (!helper) {
+    if (rounding) {
         ok = ws_round_warp(sm, bii, bk, sr, isr, ib, fqmin, fqmax);
-    } else {
+    } else if (helper) {
+        int ready = 0;   // panels of w' known to be written
         for (int d = g; d < 2 * T - 1; d += WS_GROUPS) {
             if (d >= A) {
                 // step d needs everything published up to step d-4; lane 0 waits for the warp
@@ -398,6 +533,16 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                     break;
                 }
             }
+            // step d reads w' up to column min(d, T - 1): wait for the panels that hold it
+            while (ready < min(d, T - 1) / WS_PANEL && ok) {
+                ++ready;
+                bool w_ok = true;
+                if ((tid & 31) == 0)
+                    w_ok = tc::mbar_wait(&sm.pbar[ready], 0u, WS_MAX_WAIT_CYCLES, &sm.abort_flag);
+                __syncwarp();
+                ok = __shfl_sync(0xffffffffu, (int)w_ok, 0) != 0;
+            }
+            if (!ok) break;
             const int j = d - i;
             const bool active = (unsigned)j < (unsigned)T;
             const int jr = active ? j : 0;
@@ -445,36 +590,55 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     // ---- write back: codes, V = s_i code, E (16-byte stores where the layout allows)
     constexpr int PER_ROW = T / VW;
     if (helper) {
+        // whole 4-entry runs of codes, V and E go out as one store each when the run lies inside the
+        // matrix and its addresses are aligned (the output pointers need not be)
+        const bool vec_ok = (n & 3) == 0 && ((reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(outE)) & 15) == 0 &&
+                            (reinterpret_cast<uintptr_t>(codes) & (code_bytes == 1 ? 3 : 15)) == 0;
         for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
             const int rr = f / PER_ROW, cc = (f % PER_ROW) * VW;
             const int64_t gi = r0 + rr, gj = c0 + cc;
             const float4 evv = *reinterpret_cast<const float4*>(&sm.Es[rr][cc]);
             leaf_store_split(Ebuf, Elo, gi * Np + gj, evv);
             if (gi < m) {
-                const float* es = reinterpret_cast<const float*>(&evv);
+                const int4 cv = *reinterpret_cast<const int4*>(&sm.Cs[rr][cc]);
+                const float sv = sm.s[rr];
+                const int64_t o = gi * n + gj;
+                if (vec_ok && gj + VW <= n) {
+                    if (code_bytes == 1)
+                        *reinterpret_cast<char4*>(static_cast<int8_t*>(codes) + o) =
+                            make_char4((signed char)cv.x, (signed char)cv.y, (signed char)cv.z, (signed char)cv.w);
+                    else
+                        *reinterpret_cast<int4*>(static_cast<int32_t*>(codes) + o) = cv;
+                    *reinterpret_cast<float4*>(V + o) =
+                        make_float4((float)cv.x * sv, (float)cv.y * sv, (float)cv.z * sv, (float)cv.w * sv);
+                    if (outE) *reinterpret_cast<float4*>(outE + o) = evv;
+                } else {
+                    const float* es = reinterpret_cast<const float*>(&evv);
+                    const int* cs = reinterpret_cast<const int*>(&cv);
 #pragma unroll
-                for (int u = 0; u < VW; ++u) {
-                    if (gj + u < n) {
-                        store_code(codes, code_bytes, gi * n + gj + u, sm.Cs[rr][cc + u]);
-                        V[gi * n + gj + u] = (float)sm.Cs[rr][cc + u] * sm.s[rr];
-                        if (outE) outE[gi * n + gj + u] = es[u];
+                    for (int u = 0; u < VW; ++u) {
+                        if (gj + u < n) {
+                            store_code(codes, code_bytes, o + u, cs[u]);
+                            V[o + u] = (float)cs[u] * sv;
+                            if (outE) outE[o + u] = es[u];
+                        }
                     }
                 }
             }
         }
-    }
-    // ---- the complete X = R + local X into XTg (X transposed, leading dimension Mp, split for the
-    //      tensor-core update; independent of the write-back above: no barrier between them).  The
-    //      updates read a solved tile's X only from there, so R itself is not written back.
-    for (int idx = tid; idx < T * T; idx += WS_THREADS) {
-        const int cc = idx >> 6, rr = idx & 63;
-        sm.XT[cc][rr] += sm.Rs[rr][cc];
-    }
-    __syncthreads();
-    if (helper && XTg) {
-        for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
-            const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
-            leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, *reinterpret_cast<const float4*>(&sm.XT[cc][rr]));
+        // ---- the complete X = R + local X into XTg (X transposed, leading dimension Mp, split for the
+        //      tensor-core update).  The updates read a solved tile's X only from there, so R itself is
+        //      not written back.
+        if (XTg) {
+            for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
+                const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
+                float4 x = *reinterpret_cast<const float4*>(&sm.XT[cc][rr]);
+                x.x += sm.Rp[rr][cc];
+                x.y += sm.Rp[rr + 1][cc];
+                x.z += sm.Rp[rr + 2][cc];
+                x.w += sm.Rp[rr + 3][cc];
+                leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, x);
+            }
         }
     }
 }

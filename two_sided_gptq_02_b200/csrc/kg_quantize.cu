@@ -25,6 +25,7 @@
 //               W~[I,J] -= sum_{I': I'+J in [D0,mid)} U_B[I',I]^T X[I',J]     (column chain)
 //             Both are dense GEMMs over contiguous K ranges.
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <mutex>
 #include <utility>
@@ -279,80 +280,81 @@ static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1,
 }
 
 // ---------------------------------------------------------------------------------------
-// Two-stream schedule.  Every update push(D0 | mid | D1) is split: its targets on diagonal mid --
-// all the next leaf needs -- go on the caller's stream (the critical path); its targets on
-// diagonals (mid, D1) go on a second stream, where they overlap the leaves that follow (a leaf
-// occupies at most min(Mt, Nt) SMs).  (Splitting that rest further, into pieces of 1, 2, 4, ...
-// diagonals, measured slower: the pieces run less efficiently and contend with the leaves.)  Hazards are tracked per diagonal: a bulk update targeting
-// diagonal d records an event, and the first kernel on the critical stream that touches d waits
-// for the latest such event (the bulk stream runs in order, so that covers all earlier ones).
-// Bulk updates read only sources solved before the fork event that precedes them, and they never
-// target a diagonal the critical stream has already reached.  The caller's stream waits for the
-// bulk stream at the end.
+// Schedule.  The recursion fixes which update carries each (source, target) pair of tile
+// anti-diagonals: push(D0 | mid | D1) sends sources [D0, mid) to targets [mid, D1).  Its parts are
+// needed at different times, so each push is cut into pieces; a piece (sources [s0, s1), targets
+// [t0, t1)) may start once leaf s1 - 1 is done and is due when leaf t0 starts.  The source range is
+// first halved from the old end while it is wider than kUrgentK: each half [a, h) goes to all the
+// targets at once and is free after leaf h - 1, long before it is due (background stream).  The last
+// chunk [c, mid), at most kUrgentK wide, is cut by target:
+//   near  source mid-1 -> target mid: the adjacent tiles only; the fp32 leaf of mid computes it in
+//         its set-up, in fp64 an update on the critical stream runs it between leaves mid-1 and mid;
+//   far   sources [c, mid-1) -> target mid: free one leaf before it is due, beside leaf mid-1;
+//   next  sources [c, mid) -> target mid+1: likewise beside leaf mid;     (both: urgent stream)
+//   rest  sources [c, mid) -> targets [mid+2, D1), in pieces of 2, 4, 8, ... target diagonals, each
+//         due at the leaf of its first target (soon stream).
+// Streams, by priority: critical and urgent at the device's greatest, soon in the middle,
+// background at the least, so that waiting blocks of the critical path start first on the SMs the
+// leaves leave idle.
+// Hazards: a piece waits for the leaf that completes its sources (an event per leaf on the critical
+// stream) and for the latest piece of any other stream that targets one of its diagonals (tracked
+// per diagonal and stream); a stream runs its own pieces in order.  Every piece that targets
+// diagonal d is free by leaf d-2, so it is issued before the near piece and the leaf of d, which
+// wait for it; nothing targets d after that.  Every wait binds to an event recorded by work issued earlier, so
+// the waits cannot form a cycle.  The caller's stream forks the streams at the start and waits for
+// all of them at the end (on the error path too).
 // ---------------------------------------------------------------------------------------
-struct Sched {
-    cudaStream_t crit, bulk;
-    cudaEvent_t fork;           // re-recorded before every bulk update (waits snapshot it)
-    cudaEvent_t* done;          // ring of events recorded after bulk updates, slot = seq % ndone
-    int ndone;
-    std::vector<int> pending;   // per diagonal: sequence number of the latest bulk update targeting it
-    int seq = -1;               // sequence number of the latest bulk update
-    int waited = -1;            // latest bulk update the critical stream has waited for
+enum SchedStream : int { SS_CRIT = 0, SS_URGENT = 1, SS_SOON = 2, SS_BACK = 3, SS_COUNT = 4 };
+constexpr int kUrgentK = 4;   // widest source range of the last chunk, in tile anti-diagonals
+
+struct Piece {
+    int s0, s1;   // sources: tile anti-diagonals [s0, s1)
+    int t0, t1;   // targets: tile anti-diagonals [t0, t1)
+    int stream;
 };
 
-// The critical stream is about to touch diagonals [d0, d1): wait for the latest bulk update that
-// targets one of them.  A ring slot may since have been re-recorded by a later bulk update; the
-// wait then covers that later one too, which is conservative and cannot deadlock (bulk updates
-// wait only on fork events recorded earlier on the critical stream).
-static int sched_wait(Sched& s, int d0, int d1) {
-    int need = -1;
-    for (int d = d0; d < d1; ++d) need = std::max(need, s.pending[d]);
-    if (need > s.waited) {
-        KG_CUDA_TRY(cudaStreamWaitEvent(s.crit, s.done[need % s.ndone], 0));
-        s.waited = need;
+// The pieces of push(D0 | mid | D1) other than the near one, each appended to free_at[the leaf
+// after which it may start].
+static void push_pieces(int D0, int mid, int D1, std::vector<std::vector<Piece>>& free_at) {
+    int c = D0;
+    while (mid - c > kUrgentK) {
+        const int h = (c + mid) / 2;
+        free_at[h - 1].push_back(Piece{c, h, mid, D1, SS_BACK});
+        c = h;
     }
-    return KG_OK;
+    if (c < mid - 1) free_at[mid - 2].push_back(Piece{c, mid - 1, mid, mid + 1, SS_URGENT});    // far
+    if (mid + 1 < D1) free_at[mid - 1].push_back(Piece{c, mid, mid + 1, mid + 2, SS_URGENT});   // next
+    for (int t0 = mid + 2, w = 2; t0 < D1; t0 += w, w *= 2)                                     // rest
+        free_at[mid - 1].push_back(Piece{c, mid, t0, std::min(D1, t0 + w), SS_SOON});
 }
 
-template <typename Real>
-static int solve_range(const QArgs<Real>& a, Sched& s, int D0, int D1) {
-    int rc;
-    if (D1 - D0 == 1) {
-        if ((rc = sched_wait(s, D0, D0 + 1))) return rc;
-        return launch_leaf(a, D0, s.crit);
-    }
+static void plan_pieces(int D0, int D1, std::vector<std::vector<Piece>>& free_at) {
+    if (D1 - D0 <= 1) return;
     const int mid = (D0 + D1) / 2;
-    if ((rc = solve_range(a, s, D0, mid))) return rc;
-    if ((rc = sched_wait(s, mid, mid + 1))) return rc;
-    if ((rc = launch_push(a, D0, mid, mid, mid + 1, s.crit, true))) return rc;
-    if (D1 > mid + 1) {
-        KG_CUDA_TRY(cudaEventRecord(s.fork, s.crit));
-        KG_CUDA_TRY(cudaStreamWaitEvent(s.bulk, s.fork, 0));
-        if ((rc = launch_push(a, D0, mid, mid + 1, D1, s.bulk, false))) return rc;
-        ++s.seq;
-        KG_CUDA_TRY(cudaEventRecord(s.done[s.seq % s.ndone], s.bulk));
-        for (int d = mid + 1; d < D1; ++d) s.pending[d] = s.seq;
-    }
-    return solve_range(a, s, mid, D1);
+    plan_pieces(D0, mid, free_at);
+    push_pieces(D0, mid, D1, free_at);
+    plan_pieces(mid, D1, free_at);
 }
 
-// Per host thread and device: a few bulk streams with their events, created on first use and kept
-// for the life of the process (a thread that exits leaves its slots allocated; nothing is destroyed
-// at exit, when the CUDA runtime may already be gone).  Calls take them in turn, so that solves in
-// flight at the same time on different caller streams (several layers at once) also run their bulk
-// updates side by side; two calls that share a slot only serialise their bulk work.
+// Per host thread and device: a few sets of the four streams with their events, created on first
+// use and kept for the life of the process (a thread that exits leaves its slots allocated; nothing
+// is destroyed at exit, when the CUDA runtime may already be gone).  Calls take them in turn, so
+// that solves in flight at the same time on different caller streams (several layers at once) run
+// side by side; two calls that share a slot only serialise.
+static constexpr int kSchedSlots = 8;
+static constexpr int kSchedEvents = 64;   // ring of events per stream, and one for the leaves
 struct SchedSlot {
-    cudaStream_t bulk = nullptr;
+    cudaStream_t s[SS_COUNT] = {};
     cudaEvent_t fork = nullptr;
-    std::vector<cudaEvent_t> done;
+    cudaEvent_t join[SS_COUNT] = {};
+    std::vector<cudaEvent_t> ev[SS_COUNT];
+    std::vector<cudaEvent_t> leaf_ev;
 };
 struct SchedPool {
     int dev = -1;
     unsigned next = 0;
     std::vector<SchedSlot> slots;
 };
-static constexpr int kSchedSlots = 8;
-static constexpr int kSchedDone = 64;
 
 static int sched_slot(SchedSlot*& out) {
     static thread_local std::vector<SchedPool> pools;
@@ -362,14 +364,23 @@ static int sched_slot(SchedSlot*& out) {
     for (auto& p : pools)
         if (p.dev == dev) pool = &p;
     if (!pool) {
+        int least = 0, greatest = 0;
+        KG_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
         SchedPool p;
         p.dev = dev;
         p.slots.resize(kSchedSlots);
+        auto mk = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming); };
         for (auto& sl : p.slots) {
-            KG_CUDA_TRY(cudaStreamCreateWithFlags(&sl.bulk, cudaStreamNonBlocking));
-            KG_CUDA_TRY(cudaEventCreateWithFlags(&sl.fork, cudaEventDisableTiming));
-            sl.done.resize(kSchedDone);
-            for (auto& e : sl.done) KG_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+            for (int k = 0; k < SS_COUNT; ++k) {
+                const int prio = k == SS_BACK ? least : k == SS_SOON ? (least + greatest) / 2 : greatest;
+                KG_CUDA_TRY(cudaStreamCreateWithPriority(&sl.s[k], cudaStreamNonBlocking, prio));
+                KG_CUDA_TRY(mk(&sl.join[k]));
+                sl.ev[k].resize(kSchedEvents);
+                for (auto& e : sl.ev[k]) KG_CUDA_TRY(mk(&e));
+            }
+            KG_CUDA_TRY(mk(&sl.fork));
+            sl.leaf_ev.resize(kSchedEvents);
+            for (auto& e : sl.leaf_ev) KG_CUDA_TRY(mk(&e));
         }
         pools.push_back(std::move(p));
         pool = &pools.back();
@@ -378,16 +389,109 @@ static int sched_slot(SchedSlot*& out) {
     return KG_OK;
 }
 
+struct Sched {
+    SchedSlot* sl;
+    int seq[SS_COUNT] = {-1, -1, -1, -1};              // latest piece per stream
+    int waited[SS_COUNT][SS_COUNT];                    // [S][o]: latest piece of o that S waits for
+    int leaf_waited[SS_COUNT] = {-1, -1, -1, -1};      // latest leaf that S waits for
+    std::vector<std::array<int, SS_COUNT>> pending;    // per diagonal: latest piece per stream on it
+};
+
+// Stream S is about to write targets [t0, t1): wait for the latest piece of every other stream
+// that targets one of them.  A ring slot may since have been re-recorded by a later piece of the
+// same stream; the wait then covers that one too, which is only conservative.
+static int sched_hazards(Sched& s, int S, int t0, int t1) {
+    for (int o = 0; o < SS_COUNT; ++o) {
+        if (o == S) continue;
+        int need = -1;
+        for (int t = t0; t < t1; ++t) need = std::max(need, s.pending[t][o]);
+        if (need > s.waited[S][o]) {
+            KG_CUDA_TRY(cudaStreamWaitEvent(s.sl->s[S], s.sl->ev[o][need % kSchedEvents], 0));
+            s.waited[S][o] = need;
+        }
+    }
+    return KG_OK;
+}
+
+template <typename Real>
+static int sched_piece(const QArgs<Real>& a, Sched& s, const Piece& p) {
+    const int S = p.stream;
+    int rc;
+    if (p.s1 - 1 > s.leaf_waited[S]) {
+        KG_CUDA_TRY(cudaStreamWaitEvent(s.sl->s[S], s.sl->leaf_ev[(p.s1 - 1) % kSchedEvents], 0));
+        s.leaf_waited[S] = p.s1 - 1;
+    }
+    if ((rc = sched_hazards(s, S, p.t0, p.t1))) return rc;
+    if ((rc = launch_push(a, p.s0, p.s1, p.t0, p.t1, s.sl->s[S], false))) return rc;
+    const int q = ++s.seq[S];
+    KG_CUDA_TRY(cudaEventRecord(s.sl->ev[S][q % kSchedEvents], s.sl->s[S]));
+    for (int t = p.t0; t < p.t1; ++t) s.pending[t][S] = q;
+    return KG_OK;
+}
+
+// The order in which the solve issues its work: for every leaf L, the near piece of L (L > 0), the
+// leaf itself (a Piece with stream -1 and s0 = s1 = t0 = L, t1 = L + 1), then the pieces that leaf
+// L frees, earliest due first.
+static std::vector<Piece> issue_order(int ndiag) {
+    std::vector<std::vector<Piece>> free_at(ndiag);
+    plan_pieces(0, ndiag, free_at);
+    std::vector<Piece> order;
+    for (int L = 0; L < ndiag; ++L) {
+        if (L > 0) order.push_back(Piece{L - 1, L, L, L + 1, SS_CRIT});
+        order.push_back(Piece{L, L, L, L + 1, -1});
+        std::stable_sort(free_at[L].begin(), free_at[L].end(),
+                         [](const Piece& x, const Piece& y) { return x.t0 < y.t0; });
+        order.insert(order.end(), free_at[L].begin(), free_at[L].end());
+    }
+    return order;
+}
+
+template <typename Real>
+static int solve_leaves(const QArgs<Real>& a, Sched& s, int ndiag) {
+    const std::vector<Piece> order = issue_order(ndiag);
+    cudaStream_t crit = s.sl->s[SS_CRIT];
+    int rc;
+    for (size_t k = 0; k < order.size(); ++k) {
+        const Piece& p = order[k];
+        if (p.stream == SS_CRIT) {
+            // near piece: the fp32 leaf computes it itself in its set-up; in fp64 an update kernel
+            // runs it just before the leaf (both launched back to back, programmatic launch)
+            if constexpr (sizeof(Real) == 8) {
+                if ((rc = sched_hazards(s, SS_CRIT, p.t0, p.t1))) return rc;
+                if ((rc = launch_push(a, p.s0, p.s1, p.t0, p.t1, crit, true))) return rc;
+            }
+        } else if (p.stream < 0) {
+            const int L = p.t0;
+            if ((rc = sched_hazards(s, SS_CRIT, L, L + 1))) return rc;
+            if ((rc = launch_leaf(a, L, crit))) return rc;
+            if (k + 1 < order.size() && order[k + 1].stream > 0)   // pieces freed by this leaf follow
+                KG_CUDA_TRY(cudaEventRecord(s.sl->leaf_ev[L % kSchedEvents], crit));
+        } else if ((rc = sched_piece(a, s, p))) {
+            return rc;
+        }
+    }
+    return KG_OK;
+}
+
 template <typename Real>
 static int solve_all(const QArgs<Real>& a, int ndiag) {
     SchedSlot* slot = nullptr;
     int rc = sched_slot(slot);
     if (rc) return rc;
-    Sched s{a.st, slot->bulk, slot->fork, slot->done.data(), (int)slot->done.size(), std::vector<int>(ndiag + 1, -1)};
-    rc = solve_range(a, s, 0, ndiag);
-    // join: the caller's stream waits for the last bulk update (also on the error path, so the
-    // bulk stream never runs past the caller's view of the solve)
-    if (s.seq > s.waited) KG_CUDA_TRY(cudaStreamWaitEvent(s.crit, s.done[s.seq % s.ndone], 0));
+    Sched s;
+    s.sl = slot;
+    for (auto& w : s.waited)
+        for (int& x : w) x = -1;
+    s.pending.assign(ndiag + 1, std::array<int, SS_COUNT>{-1, -1, -1, -1});
+    KG_CUDA_TRY(cudaEventRecord(slot->fork, a.st));
+    for (int k = 0; k < SS_COUNT; ++k) KG_CUDA_TRY(cudaStreamWaitEvent(slot->s[k], slot->fork, 0));
+    rc = solve_leaves(a, s, ndiag);
+    // join: the caller's stream waits for all of them (also on the error path, so that no stream runs
+    // past the caller's view of the solve)
+    for (int k = 0; k < SS_COUNT; ++k) {
+        KG_CUDA_TRY(cudaEventRecord(slot->join[k], slot->s[k]));
+        KG_CUDA_TRY(cudaStreamWaitEvent(a.st, slot->join[k], 0));
+    }
     return rc;
 }
 
@@ -880,3 +984,17 @@ extern "C" __attribute__((visibility("default"))) int kron_gptq_debug_handoff_fa
     return cudaMemcpyToSymbol(kg::g_test_handoff_fault, &v, sizeof(v)) == cudaSuccess ? 0 : KG_ERR_CUDA;
 }
 #endif
+
+extern "C" int kron_gptq_schedule_plan(int ndiag, int* out, int max_pieces) {
+    if (ndiag < 1 || max_pieces < 0) return KG_ERR_ARG;
+    int count = 0;
+    for (const Piece& p : issue_order(ndiag)) {
+        if (p.stream < 0) continue;
+        if (out && count < max_pieces) {
+            int* o = out + 5 * (int64_t)count;
+            o[0] = p.s0; o[1] = p.s1; o[2] = p.t0; o[3] = p.t1; o[4] = p.stream;
+        }
+        ++count;
+    }
+    return count;
+}
