@@ -189,7 +189,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
 
     // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i)
     {
-        const int ty = tid >> 4, tx = tid & 15;
+        const int ty = tid >> 4, tx = tid & 15;   // rows 4 ty .. 4 ty + 3; columns tx + 16 c (c < 4)
         Real acc[4][4];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
@@ -202,7 +202,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
 #pragma unroll
             for (int a = 0; a < 4; ++a) bv[a] = sm.Es[k][ty * 4 + a];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) rv[c] = sm.XT[k][tx * 4 + c];
+            for (int c = 0; c < 4; ++c) rv[c] = sm.XT[k][tx + 16 * c];   // 16 lanes on consecutive words
 #pragma unroll
             for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -212,7 +212,7 @@ k_leaf(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp,
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) sm.Ws[ty * 4 + a][tx * 4 + c] -= acc[a][c];
+            for (int c = 0; c < 4; ++c) sm.Ws[ty * 4 + a][tx + 16 * c] -= acc[a][c];
         // Es and XT start the sweep at zero (unvisited entries contribute nothing)
         for (int idx = tid; idx < T * T; idx += 256) {
             sm.Es[idx / T][idx % T] = Real(0);

@@ -51,9 +51,7 @@ constexpr int WS_GROUPS = 4;                                 // helper groups, t
 constexpr int WS_TPR = 2;                                    // helper threads per row
 constexpr int WS_GTHREADS = KG_T * WS_TPR;                   // threads per group (four warps)
 constexpr int WS_HELPERS = WS_GTHREADS * WS_GROUPS;
-constexpr int WS_PANEL = 16;                                 // columns of w' per set-up panel
-constexpr int WS_PANEL_WARPS = KG_T / WS_PANEL - 1;          // one per panel after the first
-constexpr int WS_THREADS = WS_HELPERS + 32 + 32 * WS_PANEL_WARPS;   // + the rounding warp + panel warps
+constexpr int WS_THREADS = WS_HELPERS + 32;                  // + the rounding warp
 #ifndef KG_TEST_HANDOFF_FAULT
 constexpr long long WS_MAX_WAIT_CYCLES = 50000000LL;         // ~25 ms: far beyond any hand-off
 #else
@@ -73,6 +71,8 @@ struct LeafWsSmem {
     float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
     float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
     float Ws[KG_T][S];             // w'
+    float Rs[KG_T][KG_T + 1];      // R tile as loaded, added to the local X at the end
+                                   // (stride 65: the column walk is conflict-free)
     float colc[KG_T][8];           // column j: a[j-1][j] .. a[j-5][j], 1/a[j][j], a[j][j], unused
     float pre[WS_RING][KG_T][2];   // (P, r') of row i for step d, slot d % WS_RING
     float s[KG_T], invs[KG_T];
@@ -84,12 +84,8 @@ struct LeafWsSmem {
     float Nxu[KG_T][68];           // X of tile (I-1, J): [k][j]
     float Na[KG_T][68];            // U_A[J-1, J] block: [k][j]
     float Nb[KG_T][68];            // U_B[I-1, I] block: [k][i]
-    float Nbd[KG_T][68];           // b = U_B[I, I] block, masked to its upper triangle: [k][i]
-    float Rp[KG_T][68];            // R of the tile with the near field added: [i][j]; the fold reads
-                                   // it, and the complete X adds it to the local X at the end
     uint64_t cbar[WS_RING];        // step d published (32 arrivals)
     uint64_t hbar[WS_RING];        // (P, r') of step d written (one arrival per row)
-    uint64_t pbar[WS_PANEL_WARPS + 1];   // w' of panel p written (32 arrivals; p >= 1)
     int abort_flag;
 };
 
@@ -263,7 +259,6 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     const int J = D - I;
     const int tid = threadIdx.x;
     const bool helper = tid < WS_HELPERS;
-    const bool rounding = !helper && tid < WS_HELPERS + 32;
     grid_dep_launch();
     const int64_t r0 = (int64_t)I * T, c0 = (int64_t)J * T;
 
@@ -354,9 +349,10 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                         sm.colc[c][c - 1 - r] = x[u];   // a[c-k-1][c] at k = c - 1 - r
                     }
                 } else if (tile == 1) {   // b row-major, masked to the upper triangle
-                    sm.Nbd[r][c] = (c >= r) ? x[u] : 0.f;
-                } else if (tile == 2) {   // R: the near field adds to it, the fold reads it
-                    sm.Rp[r][c] = x[u];
+                    sm.Es[r][c] = (c >= r) ? x[u] : 0.f;
+                } else if (tile == 2) {   // R: for the fold (XT) and kept for the final X (Rs)
+                    sm.XT[r][c] = x[u];
+                    sm.Rs[r][c] = x[u];
                 } else {
                     sm.Ws[r][c] = x[u];
                 }
@@ -367,119 +363,60 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             sm.s[tid] = s;
             sm.invs[tid] = 1.f / s;
         }
-        // Es and XT start the sweep at zero (unvisited entries contribute nothing)
-        for (int idx = tid; idx < T * T / VW; idx += WS_HELPERS) {
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(&sm.Es[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
-            *reinterpret_cast<float4*>(&sm.XT[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
-        }
     }
     if (tid == 0) {
         for (int k = 0; k < WS_RING; ++k) {
             tc::mbar_init(&sm.cbar[k], 32);
             tc::mbar_init(&sm.hbar[k], 2 * T);   // both steps of a pair, one arrival per row each
         }
-        for (int k = 1; k <= WS_PANEL_WARPS; ++k) tc::mbar_init(&sm.pbar[k], 32);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
-    // ---- w' = W~ - U_B[I-1, I]^T X[I-1, J] - b^T R' with R' = R + E[I, J-1] U_A[J-1, J], fp32: the
-    //      near field (the updates from the adjacent tiles of tile anti-diagonal D - 1, which no update
-    //      kernel carries) and the fold of the row chain (b^T[i][k] = b[k][i] = 0 for k > i), each entry
-    //      one chain of fused multiply-adds (R' from R over k; w' from W~ over the near terms, then
-    //      over the fold terms).  In panels of 16 columns: the helpers make panel 0 before the sweep;
-    //      panel warp p - 1 makes panel p while the sweep runs, and the helpers wait for it before the
-    //      first step that reads one of its columns.
+    // ---- near field: the updates from the adjacent tiles of tile anti-diagonal D - 1, which no
+    //      update kernel carries:
+    //        R  += E[I, J-1] U_A[J-1, J]          (threads 0-255)
+    //        W~ -= U_B[I-1, I]^T X[I-1, J]        (threads 256-511)
+    //      fp32, a 4 x 4 block per thread: rows 4 (q >> 4) .., columns 4 (q & 15) ..
     if (helper) {
-        const int pi = tid >> 3, pj = 2 * (tid & 7);   // row, first of two columns of panel 0
-        float2 rr = *reinterpret_cast<const float2*>(&sm.Rp[pi][pj]);
-        float2 ww = *reinterpret_cast<const float2*>(&sm.Ws[pi][pj]);
-        if (has_left) {
+        const int q = tid & 255, i0 = 4 * (q >> 4), j0 = 4 * (q & 15);
+        const bool xside = tid >= 256;
+        if (xside ? has_up : has_left) {
+            float2 acc[4][2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = make_float2(0.f, 0.f);
+            const float(*A)[68] = xside ? sm.Nb : sm.Nel;   // [k][i]
+            const float(*B)[68] = xside ? sm.Nxu : sm.Na;   // [k][j]
 #pragma unroll 8
             for (int k = 0; k < T; ++k) {
-                const float e = sm.Nel[k][pi];
-                rr = __ffma2_rn(make_float2(e, e), *reinterpret_cast<const float2*>(&sm.Na[k][pj]), rr);
+                const float4 av = *reinterpret_cast<const float4*>(&A[k][i0]);
+                const float4 bv = *reinterpret_cast<const float4*>(&B[k][j0]);
+                const float2 b01 = make_float2(bv.x, bv.y), b23 = make_float2(bv.z, bv.w);
+                const float ar[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    acc[u][0] = __ffma2_rn(make_float2(ar[u], ar[u]), b01, acc[u][0]);
+                    acc[u][1] = __ffma2_rn(make_float2(ar[u], ar[u]), b23, acc[u][1]);
+                }
             }
-        }
-        if (has_up) {
-#pragma unroll 8
-            for (int k = 0; k < T; ++k) {
-                const float b = -sm.Nb[k][pi];
-                ww = __ffma2_rn(make_float2(b, b), *reinterpret_cast<const float2*>(&sm.Nxu[k][pj]), ww);
-            }
-        }
-        *reinterpret_cast<float2*>(&sm.Rp[pi][pj]) = rr;
-        asm volatile("bar.sync 1, %0;" ::"n"(WS_HELPERS) : "memory");   // R' of panel 0 complete
-#pragma unroll 4
-        for (int k = 0; k <= pi; ++k) {
-            const float b = -sm.Nbd[k][pi];
-            ww = __ffma2_rn(make_float2(b, b), *reinterpret_cast<const float2*>(&sm.Rp[k][pj]), ww);
-        }
-        *reinterpret_cast<float2*>(&sm.Ws[pi][pj]) = ww;
-    } else if (!rounding) {
-        // panel warp: rows 2l, 2l + 1 of panel p
-        const int l = tid & 31, p = (tid - WS_HELPERS - 32) / 32 + 1, cb = WS_PANEL * p, ra = 2 * l;
-        float2 acc[2][WS_PANEL / 2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+            for (int u = 0; u < 4; ++u) {
+                const float o[4] = {acc[u][0].x, acc[u][0].y, acc[u][1].x, acc[u][1].y};
+                if (xside) {
+                    float4 wv = *reinterpret_cast<float4*>(&sm.Ws[i0 + u][j0]);
+                    wv.x -= o[0]; wv.y -= o[1]; wv.z -= o[2]; wv.w -= o[3];
+                    *reinterpret_cast<float4*>(&sm.Ws[i0 + u][j0]) = wv;
+                } else {
+                    float4 rv = *reinterpret_cast<float4*>(&sm.XT[i0 + u][j0]);   // R row-major in set-up
+                    rv.x += o[0]; rv.y += o[1]; rv.z += o[2]; rv.w += o[3];
+                    *reinterpret_cast<float4*>(&sm.XT[i0 + u][j0]) = rv;
 #pragma unroll
-            for (int v = 0; v < WS_PANEL / 2; ++v) acc[u][v] = *reinterpret_cast<const float2*>(&sm.Rp[ra + u][cb + 2 * v]);
-        if (has_left) {
-#pragma unroll 2
-            for (int k = 0; k < T; ++k) {
-                const float2 e = *reinterpret_cast<const float2*>(&sm.Nel[k][ra]);
-#pragma unroll
-                for (int v = 0; v < WS_PANEL / 4; ++v) {
-                    const float4 x = *reinterpret_cast<const float4*>(&sm.Na[k][cb + 4 * v]);
-                    acc[0][2 * v] = __ffma2_rn(make_float2(e.x, e.x), make_float2(x.x, x.y), acc[0][2 * v]);
-                    acc[0][2 * v + 1] = __ffma2_rn(make_float2(e.x, e.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
-                    acc[1][2 * v] = __ffma2_rn(make_float2(e.y, e.y), make_float2(x.x, x.y), acc[1][2 * v]);
-                    acc[1][2 * v + 1] = __ffma2_rn(make_float2(e.y, e.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
+                    for (int w = 0; w < 4; ++w) sm.Rs[i0 + u][j0 + w] += o[w];
                 }
             }
         }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < WS_PANEL / 2; ++v) *reinterpret_cast<float2*>(&sm.Rp[ra + u][cb + 2 * v]) = acc[u][v];
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < WS_PANEL / 2; ++v) acc[u][v] = *reinterpret_cast<const float2*>(&sm.Ws[ra + u][cb + 2 * v]);
-        if (has_up) {
-#pragma unroll 2
-            for (int k = 0; k < T; ++k) {
-                const float2 b = *reinterpret_cast<const float2*>(&sm.Nb[k][ra]);
-#pragma unroll
-                for (int v = 0; v < WS_PANEL / 4; ++v) {
-                    const float4 x = *reinterpret_cast<const float4*>(&sm.Nxu[k][cb + 4 * v]);
-                    acc[0][2 * v] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.x, x.y), acc[0][2 * v]);
-                    acc[0][2 * v + 1] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
-                    acc[1][2 * v] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.x, x.y), acc[1][2 * v]);
-                    acc[1][2 * v + 1] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
-                }
-            }
-        }
-        __syncwarp();   // R' of the whole panel (all rows, made by this warp) before the fold reads it
-#pragma unroll 2
-        for (int k = 0; k < T; ++k) {   // b[k][i] = 0 for k > i
-            const float2 b = *reinterpret_cast<const float2*>(&sm.Nbd[k][ra]);
-#pragma unroll
-            for (int v = 0; v < WS_PANEL / 4; ++v) {
-                const float4 x = *reinterpret_cast<const float4*>(&sm.Rp[k][cb + 4 * v]);
-                acc[0][2 * v] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.x, x.y), acc[0][2 * v]);
-                acc[0][2 * v + 1] = __ffma2_rn(make_float2(-b.x, -b.x), make_float2(x.z, x.w), acc[0][2 * v + 1]);
-                acc[1][2 * v] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.x, x.y), acc[1][2 * v]);
-                acc[1][2 * v + 1] = __ffma2_rn(make_float2(-b.y, -b.y), make_float2(x.z, x.w), acc[1][2 * v + 1]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int v = 0; v < WS_PANEL / 2; ++v) *reinterpret_cast<float2*>(&sm.Ws[ra + u][cb + 2 * v]) = acc[u][v];
-        tc::mbar_arrive(&sm.pbar[p]);   // every lane: its own stores are released with its arrival
     }
+    __syncthreads();
 
     // ---- per-row constants.  Helpers: U_B column of the row for k <= i-4 in registers.
     //      Rounding warp: b_ii, b[i-1][i], b[i-2][i], b[i-3][i], s_i for its two rows.
@@ -491,33 +428,65 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
 #pragma unroll
         for (int u = 0; u < VW; ++u) {
             const int k = VW * q + WS_TPR * VW * t + u;
-            breg[t][u] = (helper && k <= i - A) ? sm.Nbd[k][i] : 0.f;
+            breg[t][u] = (helper && k <= i - A) ? sm.Es[k][i] : 0.f;
         }
     float bii[2], bk[2][6], sr[2], isr[2], ib[2];
-    if (rounding) {
+    if (!helper) {
         const int l = tid & 31;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int ir = 2 * l + r;
-            bii[r] = sm.Nbd[ir][ir];
+            bii[r] = sm.Es[ir][ir];
             bk[r][0] = 0.f;
 #pragma unroll
-            for (int k = 1; k < 6; ++k) bk[r][k] = (ir >= k) ? sm.Nbd[ir - k][ir] : 0.f;
+            for (int k = 1; k < 6; ++k) bk[r][k] = (ir >= k) ? sm.Es[ir - k][ir] : 0.f;
             sr[r] = sm.s[ir];
             isr[r] = sm.invs[ir];
             ib[r] = 1.f / bii[r];
         }
     }
-    // the helpers read w' of panel 0 made by other helpers
-    if (helper) asm volatile("bar.sync 1, %0;" ::"n"(WS_HELPERS) : "memory");
+
+    // ---- fold the external row chain: w' = W~ - b^T R  (b^T[i][k] = b[k][i] = 0 for k > i);
+    //      512 threads, a 2 x 4 block each
+    {
+        const int ty = tid >> 4, tx = tid & 15;   // rows 2 ty, 2 ty + 1; columns 4 tx .. 4 tx + 3
+        float acc[2][4];
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+        if (helper) {
+            const int kmax = ty * 2 + 1;
+#pragma unroll 4
+            for (int k = 0; k <= kmax; ++k) {
+                const float2 bv = *reinterpret_cast<const float2*>(&sm.Es[k][ty * 2]);
+                const float4 rv = *reinterpret_cast<const float4*>(&sm.XT[k][tx * 4]);
+                acc[0][0] += bv.x * rv.x; acc[0][1] += bv.x * rv.y; acc[0][2] += bv.x * rv.z; acc[0][3] += bv.x * rv.w;
+                acc[1][0] += bv.y * rv.x; acc[1][1] += bv.y * rv.y; acc[1][2] += bv.y * rv.z; acc[1][3] += bv.y * rv.w;
+            }
+        }
+        __syncthreads();
+        if (helper) {
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sm.Ws[ty * 2 + a][tx * 4 + c] -= acc[a][c];
+        }
+        // Es and XT start the sweep at zero (unvisited entries contribute nothing)
+        for (int idx = tid; idx < T * T / VW; idx += WS_THREADS) {
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(&sm.Es[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
+            *reinterpret_cast<float4*>(&sm.XT[idx / PER_ROW_Z][(idx % PER_ROW_Z) * VW]) = z;
+        }
+    }
+    __syncthreads();
 
     // ---- sweep
     const float fqmin = (float)qmin, fqmax = (float)qmax;
     bool ok = true;
-    if (rounding) {
+    if (!helper) {
         ok = ws_round_warp(sm, bii, bk, sr, isr, ib, fqmin, fqmax);
-    } else if (helper) {
-        int ready = 0;   // panels of w' known to be written
+    } else {
         for (int d = g; d < 2 * T - 1; d += WS_GROUPS) {
             if (d >= A) {
                 // step d needs everything published up to step d-4; lane 0 waits for the warp
@@ -533,16 +502,6 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                     break;
                 }
             }
-            // step d reads w' up to column min(d, T - 1): wait for the panels that hold it
-            while (ready < min(d, T - 1) / WS_PANEL && ok) {
-                ++ready;
-                bool w_ok = true;
-                if ((tid & 31) == 0)
-                    w_ok = tc::mbar_wait(&sm.pbar[ready], 0u, WS_MAX_WAIT_CYCLES, &sm.abort_flag);
-                __syncwarp();
-                ok = __shfl_sync(0xffffffffu, (int)w_ok, 0) != 0;
-            }
-            if (!ok) break;
             const int j = d - i;
             const bool active = (unsigned)j < (unsigned)T;
             const int jr = active ? j : 0;
@@ -633,10 +592,10 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             for (int f = tid; f < T * PER_ROW; f += WS_HELPERS) {
                 const int cc = f / PER_ROW, rr = (f % PER_ROW) * VW;
                 float4 x = *reinterpret_cast<const float4*>(&sm.XT[cc][rr]);
-                x.x += sm.Rp[rr][cc];
-                x.y += sm.Rp[rr + 1][cc];
-                x.z += sm.Rp[rr + 2][cc];
-                x.w += sm.Rp[rr + 3][cc];
+                x.x += sm.Rs[rr][cc];
+                x.y += sm.Rs[rr + 1][cc];
+                x.z += sm.Rs[rr + 2][cc];
+                x.w += sm.Rs[rr + 3][cc];
                 leaf_store_split(XTg, XTlo, (c0 + cc) * Mp + r0 + rr, x);
             }
         }
