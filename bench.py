@@ -24,6 +24,12 @@ import sys
 import tempfile
 import time
 
+# Every recursive solve runs on four internal streams (its leaves and three streams of update pieces);
+# with the default eight hardware connections, streams of concurrent solves share queues and
+# serialise.  This must be set before the process creates its CUDA context; a value in the
+# environment wins.
+os.environ.setdefault("CUDA_DEVICE_MAX_CONNECTIONS", "32")
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)

@@ -37,7 +37,10 @@
  *     caller's stream waits for all four at the end, so each call stays one asynchronous
  *     operation on the caller's stream.  For this each host thread keeps, per device, eight sets
  *     of four non-blocking streams with their events (host-side driver objects, no device
- *     buffers), created on the first call and kept until the process exits.
+ *     buffers), created on the first call and kept until the process exits.  Solves in flight on
+ *     several caller streams at once want more than CUDA's default eight hardware connections
+ *     (CUDA_DEVICE_MAX_CONNECTIONS, set before the CUDA context exists; the Python binding defaults
+ *     it to 32): seven 4096-to-14336-wide layers in flight took 0.087 s with 8 and 0.072 s with 32.
  *   - Concurrent calls on different streams need distinct workspaces.
  *   - Status codes: 0 = success, negative = error (see kg_status).
  */

@@ -23,7 +23,15 @@ Public functions mirror the C names:
 """
 from __future__ import annotations
 
-from ._lib import (  # noqa: F401
+import os as _os
+
+# Every recursive solve runs on four internal streams; with the default eight hardware connections
+# the streams of concurrent solves share queues and serialise.  Takes effect only if set before the
+# process creates its CUDA context (importing this package first does that); a value already in the
+# environment wins.
+_os.environ.setdefault("CUDA_DEVICE_MAX_CONNECTIONS", "32")
+
+from ._lib import (  # noqa: E402,F401
     KG_F32,
     KG_F64,
     KGError,
