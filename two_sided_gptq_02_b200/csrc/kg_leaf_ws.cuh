@@ -67,7 +67,7 @@ __device__ int g_test_handoff_fault;
 
 struct LeafWsSmem {
     static constexpr int S = LeafCfg<float>::S;
-    float aT[KG_T][S];             // aT[j][k] = a[k][j] for k <= j - 4, else 0
+    float aT[KG_T][S];             // aT[j][k] = a[k][j] for k <= j - WS_AHEAD, else 0
     float Es[KG_T][S];             // errors E[i][k]; during set-up b row-major
     float XT[KG_T][S];             // XT[j][k] = X[k][j]; during set-up R row-major
     float Ws[KG_T][S];             // w'
@@ -273,9 +273,17 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
     // chain, (I-1, J) its X down the column chain
     const bool has_left = J > 0, has_up = I > 0;
     if (helper) {
-        // the four tiles in one memory round trip: 512 threads x 8 float4, two of each tile
+        // the four tiles in one memory round trip: 512 threads x 8 float4.  The factor blocks a
+        // (threads 0-255) and b (threads 256-511) as one 4 x 4 block per thread, a read down its
+        // columns so that the transposed 16-byte stores of a quarter-warp land on distinct banks; R
+        // and W~ as two float4 each.
         const float* src[4] = {UA + c0 * ldA + c0, UB + r0 * ldB + r0, R + r0 * Np + c0, Wt + r0 * Np + c0};
         const int64_t lds[4] = {ldA, ldB, Np, Np};
+        const int fq = tid & 255, fa = tid < 256;
+        const int fk = fa ? 4 * (fq & 15) : 4 * (fq >> 4);   // first row of the block
+        const int fj = fa ? 4 * (fq >> 4) : 4 * (fq & 15);   // first column
+        const float* fsrc = fa ? UA + c0 * ldA + c0 : UB + r0 * ldB + r0;
+        const int64_t fld = fa ? ldA : ldB;
         // with the factor blocks of the near field: U_A[J-1, J] and U_B[I-1, I]
         float4 v[8], nf[4];
 #pragma unroll
@@ -292,8 +300,12 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
             // the factor tiles (f < 4) do not depend on earlier kernels of the solve: they load while
             // the previous kernel finishes; R and W~ (f >= 4) only after it has
             if (f == 4) grid_dep_wait();
-            const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;   // e: vector index in the tile
-            v[f] = *reinterpret_cast<const float4*>(src[tile] + (int64_t)(e >> 4) * lds[tile] + (e & 15) * 4);
+            if (f < 4) {
+                v[f] = *reinterpret_cast<const float4*>(fsrc + (int64_t)(fk + f) * fld + fj);
+            } else {
+                const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;   // e: vector index in the tile
+                v[f] = *reinterpret_cast<const float4*>(src[tile] + (int64_t)(e >> 4) * lds[tile] + (e & 15) * 4);
+            }
         }
         // the near-field sources, written by the previous leaf: E of (I, J-1) (threads 0-255) and X^T of
         // (I-1, J) (threads 256-511), each as its two tf32 planes (hi + lo is the value to within 2^-22
@@ -332,25 +344,44 @@ k_leaf_ws(int D, int Mt, int Nt, int64_t m, int64_t n, int64_t Np, int64_t Mp, f
                 *reinterpret_cast<float4*>(&dstT[4 * (q & 15) + w][4 * (q >> 4)]) =
                     make_float4(blk[0][w], blk[1][w], blk[2][w], blk[3][w]);
         }
+        if (fa) {   // a: transposed, masked to k <= j - WS_AHEAD; the column constants
 #pragma unroll
-        for (int f = 0; f < 8; ++f) {
+            for (int w = 0; w < 4; ++w) {   // v[u] = a[fk + u][fj .. fj + 3]
+                const int c = fj + w;
+                float o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = fk + u;
+                    const float x = w == 0 ? v[u].x : w == 1 ? v[u].y : w == 2 ? v[u].z : v[u].w;
+                    o[u] = (r <= c - A) ? x : 0.f;
+                    if (r == c) {
+                        sm.colc[c][6] = x;
+                        sm.colc[c][5] = 1.f / x;
+                    } else if (r < c && r >= c - (WS_AHEAD - 1)) {
+                        sm.colc[c][c - 1 - r] = x;   // a[c-k-1][c] at k = c - 1 - r
+                    }
+                }
+                *reinterpret_cast<float4*>(&sm.aT[c][fk]) = make_float4(o[0], o[1], o[2], o[3]);
+            }
+        } else {   // b row-major, masked to the upper triangle
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = fk + u;
+                const float4 x = v[u];
+                *reinterpret_cast<float4*>(&sm.Es[r][fj]) =
+                    make_float4(fj >= r ? x.x : 0.f, fj + 1 >= r ? x.y : 0.f, fj + 2 >= r ? x.z : 0.f,
+                                fj + 3 >= r ? x.w : 0.f);
+            }
+        }
+#pragma unroll
+        for (int f = 4; f < 8; ++f) {
             const int e = (f & 1) * WS_HELPERS + tid, tile = f >> 1;
             const int r = e >> 4, c4 = (e & 15) * 4;
             const float* x = reinterpret_cast<const float*>(&v[f]);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int c = c4 + u;
-                if (tile == 0) {          // a: transposed, masked to k <= j-4; column constants
-                    sm.aT[c][r] = (r <= c - A) ? x[u] : 0.f;
-                    if (r == c) {
-                        sm.colc[c][6] = x[u];
-                        sm.colc[c][5] = 1.f / x[u];
-                    } else if (r < c && r >= c - (WS_AHEAD - 1)) {
-                        sm.colc[c][c - 1 - r] = x[u];   // a[c-k-1][c] at k = c - 1 - r
-                    }
-                } else if (tile == 1) {   // b row-major, masked to the upper triangle
-                    sm.Es[r][c] = (c >= r) ? x[u] : 0.f;
-                } else if (tile == 2) {   // R: for the fold (XT) and kept for the final X (Rs)
+                if (tile == 2) {   // R: for the fold (XT) and kept for the final X (Rs)
                     sm.XT[r][c] = x[u];
                     sm.Rs[r][c] = x[u];
                 } else {
