@@ -87,7 +87,9 @@ __device__ __forceinline__ Real leaf_clamp(Real v, Real lo, Real hi) {
 
 // Copy four 64x64 tiles of row-major matrices into shared memory with a per-element transform
 // store(tile, r, c, x), in PASSES memory round trips: each pass issues its share of the global
-// loads of all four tiles before any store.  Threads 0..255 take part.
+// loads of all four tiles before any store.  Threads 0..255 take part.  Tile 0, which the store
+// transposes, is taken down its columns (a warp's lanes on consecutive rows), so that the transposed
+// stores of a warp land on consecutive words; the others along their rows.
 template <typename Real, int PASSES, class Store>
 __device__ __forceinline__ void leaf_load_tiles4(const Real* const (&src)[4], const int64_t (&ld)[4], Store store) {
     constexpr int VW = LeafCfg<Real>::VW;
@@ -103,7 +105,7 @@ __device__ __forceinline__ void leaf_load_tiles4(const Real* const (&src)[4], co
 #pragma unroll
             for (int e = 0; e < PER_PASS; ++e) {
                 const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
-                const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+                const int r = t == 0 ? f % KG_T : f / PER_ROW, c = (t == 0 ? f / KG_T : f % PER_ROW) * VW;
                 v[t][e] = *reinterpret_cast<const Vec*>(src[t] + (int64_t)r * ld[t] + c);
             }
 #pragma unroll
@@ -111,7 +113,7 @@ __device__ __forceinline__ void leaf_load_tiles4(const Real* const (&src)[4], co
 #pragma unroll
             for (int e = 0; e < PER_PASS; ++e) {
                 const int f = (p * PER_PASS + e) * 256 + threadIdx.x;
-                const int r = f / PER_ROW, c = (f % PER_ROW) * VW;
+                const int r = t == 0 ? f % KG_T : f / PER_ROW, c = (t == 0 ? f / KG_T : f % PER_ROW) * VW;
                 const Real* x = reinterpret_cast<const Real*>(&v[t][e]);
 #pragma unroll
                 for (int u = 0; u < VW; ++u) store(t, r, c + u, x[u]);
