@@ -771,7 +771,9 @@ def run_ours(args, rank, world, local_rank):
                 hcodes[b].copy_(qs[b].codes, non_blocking=True)
             ev_out[b].record(d2h)
 
-        for k in range(nb):
+        # warm-up: twice per input set, so that the library's capture of each set's solve into a CUDA
+        # graph (on the second call with the same arguments) happens before the timed region
+        for k in range(2 * nb):
             e2e_step(k)
         torch.cuda.synchronize()
         barrier()

@@ -66,3 +66,39 @@ def test_graph_replay_matches_direct_solve(kg, dtype, m, n):
     assert torch.equal(got[2], ref_E)
     # and the replay solved the new W, not the one present at capture
     assert not torch.equal(got[0], codes_before)
+
+
+@pytest.mark.parametrize("dtype,m,n", [(torch.float32, 640, 768), (torch.float32, 200, 330),
+                                       (torch.float64, 448, 320)])
+def test_repeated_calls_replay_the_same_solve(kg, dtype, m, n):
+    """kron_gptq_quantize (fp32) captures the second call with the same arguments into a graph and
+    replays it from the third on; fp64 always runs directly.  Every call must give what a first call on fresh buffers gives (always run
+    directly), with W changed in place between calls, and the launch counters must grow by the same
+    amount per call whichever way it ran."""
+    spec, (W, A, B) = small_layer(m, n, 29, bits=3)
+    npd = np.float64 if dtype == torch.float64 else np.float32
+    UA = torch.from_numpy(oracle.prepare_lapack(A.numpy(), 0.01).astype(npd)).cuda()
+    UB = torch.from_numpy(oracle.prepare_lapack(B.numpy(), 0.01).astype(npd)).cuda()
+    Wd = torch.from_numpy(W.numpy().astype(npd)).cuda()
+    sd = kg.kron_gptq_row_scales(Wd, spec.qmax)
+    q = kg.Quantizer(m, n, dtype, Wd.device, want_E=True)
+    gen = torch.Generator(device="cpu").manual_seed(11)
+    per_call = []
+    for call in range(4):
+        if call >= 2:   # a new W under the same pointer
+            Wd.mul_(1.0 + 0.05 * torch.randn(m, n, generator=gen, dtype=torch.float64).to(dtype).cuda())
+            sd.copy_(kg.kron_gptq_row_scales(Wd, spec.qmax))
+        kg.kron_gptq_profile_read(reset=True)
+        q.codes.fill_(99)
+        q.run(Wd, UA, UB, sd, spec.qmin, spec.qmax)
+        torch.cuda.synchronize()
+        counts = kg.kron_gptq_profile_read(reset=True)
+        per_call.append(sum(v[0] for v in counts.values()))
+        assert q.status() == 0
+        fresh = kg.Quantizer(m, n, dtype, Wd.device, want_E=True)   # new buffers: a first call, direct
+        fresh.run(Wd, UA, UB, sd, spec.qmin, spec.qmax)
+        assert fresh.status() == 0
+        assert torch.equal(q.codes, fresh.codes), f"call {call}"
+        assert torch.equal(q.V, fresh.V), f"call {call}"
+        assert torch.equal(q.E, fresh.E), f"call {call}"
+    assert len(set(per_call)) == 1 and per_call[0] > 0, per_call

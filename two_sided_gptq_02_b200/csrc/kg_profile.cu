@@ -51,6 +51,16 @@ void prof_after(int kind, cudaStream_t st) {
     t_open = nullptr;
 }
 
+bool prof_timing() { return g_enabled.load(std::memory_order_relaxed) != 0; }
+
+void prof_counts(int64_t out[PK_COUNT]) {
+    for (int k = 0; k < PK_COUNT; ++k) out[k] = g_launches[k].load(std::memory_order_relaxed);
+}
+
+void prof_add(const int64_t add[PK_COUNT]) {
+    for (int k = 0; k < PK_COUNT; ++k) g_launches[k].fetch_add(add[k], std::memory_order_relaxed);
+}
+
 }  // namespace kg
 
 using namespace kg;

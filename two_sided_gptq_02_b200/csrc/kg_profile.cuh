@@ -23,6 +23,9 @@ enum ProfKind : int {
 // Host-side profiler state (defined in kg_profile.cu).
 void prof_before(int kind, cudaStream_t st);
 void prof_after(int kind, cudaStream_t st);
+bool prof_timing();                          // event timing on (kron_gptq_profile_enable)
+void prof_counts(int64_t out[PK_COUNT]);     // launches counted so far, per kind
+void prof_add(const int64_t add[PK_COUNT]);  // count launches made by a graph replay
 
 struct ProfScope {
     int kind;
