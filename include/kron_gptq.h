@@ -245,6 +245,7 @@ KG_API int kron_gptq_quantize_noalloc(const void* W, int64_t m, int64_t n, int d
  * m == 0 or n == 0 is a no-op returning KG_OK.
  * Device errors: KG_ERR_NONFINITE (NaN/Inf in W, a step not finite and > 0, a factor diagonal
  *   not > 0), KG_ERR_RANGE, KG_ERR_TIMEOUT.
+ * Replays: as kron_gptq_quantize (fp32, up to 160 tile anti-diagonals, same arguments again).
  * --------------------------------------------------------------------------------------- */
 KG_API size_t kron_gptq_quantize_rc_workspace_size(int64_t m, int64_t n, int dtype);
 KG_API int kron_gptq_quantize_rc(const void* W, int64_t m, int64_t n, int dtype,

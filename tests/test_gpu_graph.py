@@ -102,3 +102,28 @@ def test_repeated_calls_replay_the_same_solve(kg, dtype, m, n):
         assert torch.equal(q.V, fresh.V), f"call {call}"
         assert torch.equal(q.E, fresh.E), f"call {call}"
     assert len(set(per_call)) == 1 and per_call[0] > 0, per_call
+
+
+def test_repeated_rc_calls_replay_the_same_solve(kg):
+    """The scaled-alphabet call (kron_gptq_quantize_rc) is replayed the same way: every call equals
+    a first call on fresh buffers, with W changed in place between calls."""
+    m, n = 384, 512
+    spec, (W, A, B) = small_layer(m, n, 31, bits=3)
+    UA = torch.from_numpy(oracle.prepare_lapack(A.numpy(), 0.01).astype(np.float32)).cuda()
+    UB = torch.from_numpy(oracle.prepare_lapack(B.numpy(), 0.01).astype(np.float32)).cuda()
+    Wd = torch.from_numpy(W.numpy().astype(np.float32)).cuda()
+    alpha, beta = kg.kron_gptq_waterkron_scales(UA, UB, 0.05)
+    q = kg.RcQuantizer(m, n, torch.float32, Wd.device, want_E=True)
+    gen = torch.Generator(device="cpu").manual_seed(13)
+    for call in range(4):
+        if call >= 2:
+            Wd.mul_(1.0 + 0.05 * torch.randn(m, n, generator=gen).cuda())
+        q.Z.fill_(12345)
+        q.run(Wd, UA, UB, alpha, beta)
+        assert q.status() == 0
+        fresh = kg.RcQuantizer(m, n, torch.float32, Wd.device, want_E=True)
+        fresh.run(Wd, UA, UB, alpha, beta)
+        assert fresh.status() == 0
+        assert torch.equal(q.Z, fresh.Z), f"call {call}"
+        assert torch.equal(q.V, fresh.V), f"call {call}"
+        assert torch.equal(q.E, fresh.E), f"call {call}"

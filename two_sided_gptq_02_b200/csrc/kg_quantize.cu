@@ -664,7 +664,8 @@ extern "C" size_t kron_gptq_quantize_workspace_size(int64_t m, int64_t n, int dt
 // of the piece streams, and such a wait keeps a leaf from starting early while the previous leaf
 // finishes; captured into a CUDA graph, the same work keeps its programmatic edges beside the
 // ordinary ones (4096^2 fp32: 7.14 -> 6.71 ms a solve, bit-identical results).  So
-// kron_gptq_quantize replays a captured graph when the same arguments come back on the same device:
+// kron_gptq_quantize (and kron_gptq_quantize_rc, whose solve is the same) replays a captured graph
+// when the same arguments come back on the same device:
 // the first call with a given set runs directly, the second is captured (on a stream of the
 // library's own: the caller's may be the legacy default stream, which cannot capture) and launched
 // on the caller's stream, later ones replay it there.  fp32 only (the fp64 solve, whose leaves take
@@ -679,11 +680,9 @@ extern "C" size_t kron_gptq_quantize_workspace_size(int64_t m, int64_t n, int dt
 constexpr int kGraphMaxDiag = 160;
 constexpr int kGraphCache = 32;
 
-struct GraphKey {   // every argument that shapes the launches (zero-filled first: compared bytewise)
-    const void *W, *UA, *UB, *scale, *codes, *V, *E, *ws;
-    int64_t m, n;
-    size_t ws_bytes;
-    int dtype, qmin, qmax, dev;
+// Every argument that shapes a call's launches, as words (zero-filled first: compared bytewise).
+struct GraphKey {
+    uint64_t w[16];
 };
 struct GraphEntry {
     GraphKey key;
@@ -700,6 +699,92 @@ static bool graphs_allowed() {
     }();
     return on;
 }
+
+// Run a call whose launches run(s) issues on stream s: directly, or as a replay of the graph captured
+// the second time the same key came, per the rules above.  eligible: the call's own conditions
+// (dtype and size) allow a replay.
+template <class Run>
+static int run_replayed(GraphKey key, bool eligible, cudaStream_t st, Run run) {
+    if (!eligible || !graphs_allowed() || prof_timing()) return run(st);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    KG_CUDA_TRY(cudaStreamIsCapturing(st, &cap));
+    if (cap != cudaStreamCaptureStatusNone) return run(st);
+    int dev = 0;
+    KG_CUDA_TRY(cudaGetDevice(&dev));
+    key.w[15] = (uint64_t)dev;
+
+    static thread_local std::vector<GraphEntry> cache;
+    static thread_local uint64_t clock = 0;
+    GraphEntry* e = nullptr;
+    for (auto& c : cache)
+        if (std::memcmp(&c.key, &key, sizeof(key)) == 0) e = &c;
+    if (!e) {   // first call with these arguments: run it directly and remember it
+        if ((int)cache.size() >= kGraphCache) {
+            auto lru = std::min_element(cache.begin(), cache.end(), [](const GraphEntry& x, const GraphEntry& y) {
+                return x.last_use < y.last_use;
+            });
+            if (lru->exec) {
+                // a replay of it may still run on some stream: let the device finish before destroying it
+                KG_CUDA_TRY(cudaDeviceSynchronize());
+                cudaGraphExecDestroy(lru->exec);
+            }
+            cache.erase(lru);
+        }
+        GraphEntry fresh;
+        std::memset(&fresh, 0, sizeof(fresh));
+        fresh.key = key;
+        fresh.last_use = ++clock;
+        cache.push_back(fresh);
+        return run(st);
+    }
+    e->last_use = ++clock;
+    if (e->exec) {   // replay
+        KG_CUDA_TRY(cudaGraphLaunch(e->exec, st));
+        prof_add(e->launches);
+        return KG_OK;
+    }
+    if (e->no_graph) return run(st);
+
+    // second call: capture on the library's capture stream, then launch on the caller's
+    static thread_local std::vector<std::pair<int, cudaStream_t>> cap_streams;   // per device
+    cudaStream_t cs = nullptr;
+    for (auto& d : cap_streams)
+        if (d.first == dev) cs = d.second;
+    if (!cs) {
+        KG_CUDA_TRY(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+        cap_streams.emplace_back(dev, cs);
+    }
+    int64_t before[PK_COUNT], after[PK_COUNT];
+    prof_counts(before);
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        (void)cudaGetLastError();
+        e->no_graph = true;
+        return run(st);
+    }
+    const int rc = run(cs);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t end = cudaStreamEndCapture(cs, &graph);
+    prof_counts(after);
+    for (int k = 0; k < PK_COUNT; ++k) e->launches[k] = after[k] - before[k];
+    cudaGraphExec_t exec = nullptr;
+    const bool ok = rc == KG_OK && end == cudaSuccess && graph &&
+                    cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    if (!ok) {   // nothing ran: take the captured launches back out of the counts and run directly
+        (void)cudaGetLastError();
+        int64_t back[PK_COUNT];
+        for (int k = 0; k < PK_COUNT; ++k) back[k] = -e->launches[k];
+        prof_add(back);
+        e->no_graph = true;
+        if (rc != KG_OK) return rc;
+        return run(st);
+    }
+    e->exec = exec;
+    KG_CUDA_TRY(cudaGraphLaunch(exec, st));   // the captured launches were counted once already
+    return KG_OK;
+}
+
+static uint64_t kw(const void* p) { return (uint64_t)reinterpret_cast<uintptr_t>(p); }
 
 static int quantize_direct(const void* W, int64_t m, int64_t n, int dtype, const void* U_A, const void* U_B,
                            kg_grid grid, int8_t* out_codes, void* out_V, void* out_E, void* ws, size_t ws_bytes,
@@ -732,91 +817,15 @@ extern "C" int kron_gptq_quantize(const void* W, int64_t m, int64_t n, int dtype
     if (ws_bytes < q_layout(m, n, dtype == KG_F64 ? 8 : 4).total) return KG_ERR_WORKSPACE;
 
     const int64_t ndiag = ceil_div(m, (int64_t)KG_T) + ceil_div(n, (int64_t)KG_T) - 1;
-    if (dtype != KG_F32 || !graphs_allowed() || prof_timing() || ndiag > kGraphMaxDiag)
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    KG_CUDA_TRY(cudaStreamIsCapturing(st, &cap));
-    if (cap != cudaStreamCaptureStatusNone)
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-
     GraphKey key;
     std::memset(&key, 0, sizeof(key));
-    key.W = W; key.UA = U_A; key.UB = U_B; key.scale = grid.row_scale;
-    key.codes = out_codes; key.V = out_V; key.E = out_E; key.ws = ws;
-    key.m = m; key.n = n; key.ws_bytes = ws_bytes;
-    key.dtype = dtype; key.qmin = grid.qmin; key.qmax = grid.qmax;
-    KG_CUDA_TRY(cudaGetDevice(&key.dev));
-
-    static thread_local std::vector<GraphEntry> cache;
-    static thread_local uint64_t clock = 0;
-    GraphEntry* e = nullptr;
-    for (auto& c : cache)
-        if (std::memcmp(&c.key, &key, sizeof(key)) == 0) e = &c;
-    if (!e) {   // first call with these arguments: run it directly and remember it
-        if ((int)cache.size() >= kGraphCache) {
-            auto lru = std::min_element(cache.begin(), cache.end(), [](const GraphEntry& a, const GraphEntry& b) {
-                return a.last_use < b.last_use;
-            });
-            if (lru->exec) {
-                // a replay of it may still run on some stream: let the device finish before destroying it
-                KG_CUDA_TRY(cudaDeviceSynchronize());
-                cudaGraphExecDestroy(lru->exec);
-            }
-            cache.erase(lru);
-        }
-        GraphEntry fresh;
-        std::memset(&fresh, 0, sizeof(fresh));
-        fresh.key = key;
-        fresh.last_use = ++clock;
-        cache.push_back(fresh);
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-    }
-    e->last_use = ++clock;
-    if (e->exec) {   // replay
-        KG_CUDA_TRY(cudaGraphLaunch(e->exec, st));
-        prof_add(e->launches);
-        return KG_OK;
-    }
-    if (e->no_graph)
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-
-    // second call: capture the solve on the library's capture stream, then launch it on the caller's
-    static thread_local std::vector<std::pair<int, cudaStream_t>> cap_streams;   // per device
-    cudaStream_t cs = nullptr;
-    for (auto& d : cap_streams)
-        if (d.first == key.dev) cs = d.second;
-    if (!cs) {
-        KG_CUDA_TRY(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
-        cap_streams.emplace_back(key.dev, cs);
-    }
-    int64_t before[PK_COUNT], after[PK_COUNT];
-    prof_counts(before);
-    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
-        (void)cudaGetLastError();
-        e->no_graph = true;
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-    }
-    const int rc = quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, cs);
-    cudaGraph_t graph = nullptr;
-    const cudaError_t end = cudaStreamEndCapture(cs, &graph);
-    prof_counts(after);
-    for (int k = 0; k < PK_COUNT; ++k) e->launches[k] = after[k] - before[k];
-    cudaGraphExec_t exec = nullptr;
-    const bool ok = rc == KG_OK && end == cudaSuccess && graph &&
-                    cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
-    if (graph) cudaGraphDestroy(graph);
-    if (!ok) {   // nothing ran: take the captured launches back out of the counts and run directly
-        (void)cudaGetLastError();
-        int64_t back[PK_COUNT];
-        for (int k = 0; k < PK_COUNT; ++k) back[k] = -e->launches[k];
-        prof_add(back);
-        e->no_graph = true;
-        if (rc != KG_OK) return rc;
-        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, st);
-    }
-    e->exec = exec;
-    KG_CUDA_TRY(cudaGraphLaunch(exec, st));   // the captured launches were counted once already
-    return KG_OK;
+    const uint64_t w[] = {1, kw(W), kw(U_A), kw(U_B), kw(grid.row_scale), kw(out_codes), kw(out_V), kw(out_E),
+                          kw(ws), (uint64_t)m, (uint64_t)n, (uint64_t)ws_bytes, (uint64_t)dtype,
+                          (uint64_t)(uint32_t)grid.qmin, (uint64_t)(uint32_t)grid.qmax};
+    std::memcpy(key.w, w, sizeof(w));
+    return run_replayed(key, dtype == KG_F32 && ndiag <= kGraphMaxDiag, st, [&](cudaStream_t s) {
+        return quantize_direct(W, m, n, dtype, U_A, U_B, grid, out_codes, out_V, out_E, ws, ws_bytes, s);
+    });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -995,14 +1004,22 @@ extern "C" int kron_gptq_quantize_rc(const void* W, int64_t m, int64_t n, int dt
     }
     if (!W || !U_A || !U_B || !alpha || !beta || !out_Z || !out_V) return KG_ERR_ARG;
     if (ws_bytes < rc_layout(m, n, dtype == KG_F64 ? 8 : 4).total) return KG_ERR_WORKSPACE;
-    if (dtype == KG_F64) {
-        int rc = configure_leaf<double>();
+    const int64_t ndiag = ceil_div(m, (int64_t)KG_T) + ceil_div(n, (int64_t)KG_T) - 1;
+    GraphKey key;   // replayed as kron_gptq_quantize is
+    std::memset(&key, 0, sizeof(key));
+    const uint64_t w[] = {2, kw(W), kw(U_A), kw(U_B), kw(alpha), kw(beta), kw(out_Z), kw(out_V), kw(out_E),
+                          kw(ws), (uint64_t)m, (uint64_t)n, (uint64_t)ws_bytes, (uint64_t)dtype};
+    std::memcpy(key.w, w, sizeof(w));
+    return run_replayed(key, dtype == KG_F32 && ndiag <= kGraphMaxDiag, st, [&](cudaStream_t s) {
+        if (dtype == KG_F64) {
+            int rc = configure_leaf<double>();
+            if (rc) return rc;
+            return quantize_rc_impl<double>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, s);
+        }
+        int rc = configure_leaf<float>();
         if (rc) return rc;
-        return quantize_rc_impl<double>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, st);
-    }
-    int rc = configure_leaf<float>();
-    if (rc) return rc;
-    return quantize_rc_impl<float>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, st);
+        return quantize_rc_impl<float>(W, m, n, U_A, U_B, alpha, beta, out_Z, out_V, out_E, ws, s);
+    });
 }
 
 extern "C" int kron_gptq_waterkron_scales(const void* U_A, int64_t n, const void* U_B, int64_t m, int dtype,
