@@ -31,6 +31,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kg_common.cuh"
@@ -65,6 +66,16 @@ struct PushCfg {
 };
 // the band (in K tiles) from which the update pairs operand tiles
 constexpr int PUSH_PAIR_MIN_K = 4;
+
+// Grid of k_push_tc32<2> for targets on diagonals [tgt0, D1): x = the operand pairs around one
+// target pair (at most (D1 - tgt0 + 2) / 2 + 1 of them), y = target pair slots j from the lowest
+// to the highest that a CTA with work can take, z = chain.
+inline dim3 push_grid_tmajor(int tgt0, int D1, int Mt, int Nt) {
+    const int gx = (std::max(Mt, Nt) + 1) / 2;
+    const int j0 = std::max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1;
+    const int j1 = (std::min(std::max(Mt, Nt), D1) + 1) >> 1;
+    return dim3((D1 - tgt0 + 2) / 2 + 1, std::max(1, j1 - j0), 2);
+}
 
 // Split operand planes of the tensor-core update (all fp32 values exactly representable as
 // tf32).  E* are Mp x Np (row-major), XT* Np x Mp, UAT* Np x Np, UBT* Mp x Mp.
@@ -119,11 +130,27 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     // two K ranges; a B box outside its own range is loaded from beyond the tensor (zeros).
     const int chain = blockIdx.z;
     const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
-    const int b0 = NB * blockIdx.x;
+    int b0, t0;
+    if constexpr (NB == 2 && MT == 2) {
+        // Target-major order (grid from push_grid_tmajor): blockIdx.y = j picks a pair of target
+        // tiles, t0 = 2j + p where the pair starts one below the band edge of operand pair b0
+        // (p = (tgt0 - 1) mod 2), t0 = 2j where that edge is clipped to 0; blockIdx.x walks the
+        // operand pairs whose band contains it.  CTAs that run together then share their U^T row
+        // slab (operand A), the larger operand of a tall or wide layer, instead of each reading
+        // its own; the set of CTAs that do work is the one of the plain (b0, t0) order.
+        const int gx = (max(Mt, Nt) + 1) / 2;
+        const int p = (tgt0 - 1) & 1;
+        const int j = (max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1) + (int)blockIdx.y;
+        const int e = tgt0 - 1 - p - 2 * j;
+        b0 = 2 * ((e > 0 ? (e + 1) >> 1 : 0) + (int)blockIdx.x);
+        t0 = tgt0 - b0 - 1 > 0 ? p + 2 * j : 2 * j;
+    } else {
+        b0 = NB * blockIdx.x;
+        t0 = max(0, tgt0 - b0 - (NB - 1)) + MT * blockIdx.y;
+    }
     if (b0 >= Bmax) return;
     const int tlo = max(0, tgt0 - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
-    const int t0 = tlo + MT * blockIdx.y;
-    if (t0 >= thi) return;
+    if (t0 < tlo || t0 >= thi) return;
     const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
     if (k0 >= k1) return;
     grid_dep_launch();
