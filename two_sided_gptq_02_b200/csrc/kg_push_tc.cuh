@@ -68,8 +68,8 @@ struct PushCfg {
 constexpr int PUSH_PAIR_MIN_K = 4;
 
 // Grid of k_push_tc32<2> for targets on diagonals [tgt0, D1): x = the operand pairs around one
-// target pair (at most (D1 - tgt0 + 2) / 2 + 1 of them), y = target pair slots j from the lowest
-// to the highest that a CTA with work can take, z = chain.
+// target pair (at most (D1 - tgt0 + 2) / 2 + 1 of them), y = target pair slots j, from the highest
+// that a CTA with work can take down to the lowest, z = chain.
 inline dim3 push_grid_tmajor(int tgt0, int D1, int Mt, int Nt) {
     const int gx = (std::max(Mt, Nt) + 1) / 2;
     const int j0 = std::max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1;
@@ -132,15 +132,18 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
     int b0, t0;
     if constexpr (NB == 2 && MT == 2) {
-        // Target-major order (grid from push_grid_tmajor): blockIdx.y = j picks a pair of target
-        // tiles, t0 = 2j + p where the pair starts one below the band edge of operand pair b0
-        // (p = (tgt0 - 1) mod 2), t0 = 2j where that edge is clipped to 0; blockIdx.x walks the
+        // Target-major order (grid from push_grid_tmajor): blockIdx.y picks a slot j, a pair of
+        // target tiles, t0 = 2j + p where the pair starts one below the band edge of operand pair
+        // b0 (p = (tgt0 - 1) mod 2), t0 = 2j where that edge is clipped to 0; blockIdx.x walks the
         // operand pairs whose band contains it.  CTAs that run together then share their U^T row
         // slab (operand A), the larger operand of a tall or wide layer, instead of each reading
-        // its own; the set of CTAs that do work is the one of the plain (b0, t0) order.
+        // its own; the set of CTAs that do work is the one of the plain (b0, t0) order.  Slots run
+        // from the highest j down: only the high slots reach the low operand pairs, whose K ranges
+        // ([D0 - b, mid - b)) are the longest, so the longest CTAs start first and the launch
+        // ends evenly.
         const int gx = (max(Mt, Nt) + 1) / 2;
         const int p = (tgt0 - 1) & 1;
-        const int j = (max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1) + (int)blockIdx.y;
+        const int j = (max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1) + (int)(gridDim.y - 1 - blockIdx.y);
         const int e = tgt0 - 1 - p - 2 * j;
         b0 = 2 * ((e > 0 ? (e + 1) >> 1 : 0) + (int)blockIdx.x);
         t0 = tgt0 - b0 - 1 > 0 ? p + 2 * j : 2 * j;
