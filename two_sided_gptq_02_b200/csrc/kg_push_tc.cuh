@@ -67,14 +67,75 @@ struct PushCfg {
 // the band (in K tiles) from which the update pairs operand tiles
 constexpr int PUSH_PAIR_MIN_K = 4;
 
-// Grid of k_push_tc32<2> for targets on diagonals [tgt0, D1): x = the operand pairs around one
-// target pair (at most (D1 - tgt0 + 2) / 2 + 1 of them), y = target pair slots j, from the highest
-// that a CTA with work can take down to the lowest, z = chain.
-inline dim3 push_grid_tmajor(int tgt0, int D1, int Mt, int Nt) {
-    const int gx = (std::max(Mt, Nt) + 1) / 2;
-    const int j0 = std::max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1;
-    const int j1 = (std::min(std::max(Mt, Nt), D1) + 1) >> 1;
-    return dim3((D1 - tgt0 + 2) / 2 + 1, std::max(1, j1 - j0), 2);
+// Launch shapes of the update of targets on tile diagonals [tgt0, D1) from sources on [D0, mid).
+// The variant: pairs of operand tiles (NB = 2, MT = 2) for bands of PUSH_PAIR_MIN_K K tiles or more
+// with several target diagonals; one operand and one target tile per CTA (NB = 1, MT = 1, M = 64)
+// for a single target diagonal, where beside a target there is never a second one to fill M = 128;
+// otherwise one operand tile and a pair of targets (NB = 1, MT = 2).
+enum PushVariant { PV_PAIR = 0, PV_SINGLE = 1, PV_NARROW = 2 };
+__host__ __device__ inline int push_variant(int D0, int mid, int tgt0, int D1) {
+    if (mid - D0 >= PUSH_PAIR_MIN_K && D1 - tgt0 > 1) return PV_PAIR;
+    return D1 - tgt0 == 1 ? PV_SINGLE : PV_NARROW;
+}
+__host__ __device__ inline int push_imax(int a, int b) { return a > b ? a : b; }
+__host__ __device__ inline int push_imin(int a, int b) { return a < b ? a : b; }
+
+// Grid (x, y, z = chain) of a launch of the given variant.  PV_PAIR runs in target-major order:
+// x = the operand pairs around one target pair (at most (D1 - tgt0 + 2) / 2 + 1 of them), y =
+// target pair slots j, from the highest that a CTA with work can take down to the lowest.  The
+// other variants: x = operand tile, y = target pair (or the one target) above the band's edge.
+inline dim3 push_grid(int variant, int tgt0, int D1, int Mt, int Nt) {
+    const int mx = std::max(Mt, Nt);
+    if (variant == PV_PAIR) {
+        const int gx = (mx + 1) / 2;
+        const int j0 = std::max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1;
+        const int j1 = (std::min(mx, D1) + 1) >> 1;
+        return dim3((D1 - tgt0 + 2) / 2 + 1, std::max(1, j1 - j0), 2);
+    }
+    if (variant == PV_SINGLE) return dim3(mx, 1, 2);
+    return dim3(mx, (D1 - tgt0 + 1) / 2, 2);
+}
+
+// The CTA (bx, by) of chain `chain` in a launch of ny target slots (the grid's y): its operand tiles
+// b0 .. b0 + NB - 1, its target tiles t0 .. t0 + MT - 1 and its K tiles [k0, k1); false when it has
+// no work.
+//   chain 1 (column chain, into W~): b = column J (B = X^T rows), t = row I (A = U_B^T rows), K over
+//     rows I' of the source band.  chain 0 (row chain, into R, computed transposed): b = row I
+//     (B = E rows), t = column J (A = U_A^T rows), K over columns J'.
+// Tile (t, b) is a target when t + b lies in [tgt0, D1) (tgt0 >= mid: the band may be updated in
+// parts); operand tile b uses K tiles [D0 - b, mid - b).  A CTA runs over the union of its operand
+// tiles' K ranges; a B box outside its own tile's range is loaded from beyond the tensor (zeros).
+// NB = MT = 2 (target-major order): slot j is a pair of target tiles, t0 = 2j + p where the pair
+// starts one below the band edge of operand pair b0 (p = (tgt0 - 1) mod 2), t0 = 2j where that edge
+// is clipped to 0; bx walks the operand pairs whose band contains it.  CTAs that run together then
+// share their U^T row slab (operand A), the larger operand of a tall or wide layer, instead of each
+// reading its own; the CTAs with work are those of the plain (b0, t0) order of the other variants.
+// Slots run from the highest j down: only the high slots reach the low operand pairs, whose K ranges
+// are the longest, so the longest CTAs start first and the launch ends evenly.
+struct PushCta {
+    int b0, t0, k0, k1;
+};
+template <int NB, int MT>
+__host__ __device__ inline bool push_cta(int bx, int by, int ny, int chain, int D0, int mid, int tgt0, int D1,
+                                         int Mt, int Nt, PushCta& c) {
+    const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
+    if (NB == 2 && MT == 2) {
+        const int gx = (push_imax(Mt, Nt) + 1) / 2;
+        const int p = (tgt0 - 1) & 1;
+        const int j = (push_imax(0, tgt0 - 1 - 2 * (gx - 1)) >> 1) + (ny - 1 - by);
+        const int e = tgt0 - 1 - p - 2 * j;
+        c.b0 = 2 * ((e > 0 ? (e + 1) >> 1 : 0) + bx);
+        c.t0 = tgt0 - c.b0 - 1 > 0 ? p + 2 * j : 2 * j;
+    } else {
+        c.b0 = NB * bx;
+        c.t0 = push_imax(0, tgt0 - c.b0 - (NB - 1)) + MT * by;
+    }
+    if (c.b0 >= Bmax) return false;
+    const int tlo = push_imax(0, tgt0 - c.b0 - (NB - 1)), thi = push_imin(Tmax, D1 - c.b0);
+    if (c.t0 < tlo || c.t0 >= thi) return false;
+    c.k0 = push_imax(0, D0 - c.b0 - (NB - 1));
+    c.k1 = push_imin(Kmax, mid - c.b0);
+    return c.k0 < c.k1;
 }
 
 // Split operand planes of the tensor-core update (all fp32 values exactly representable as
@@ -122,40 +183,13 @@ k_push_tc32(int D0, int mid, int tgt0, int D1, int Mt, int Nt, int64_t Np, float
     int* issued_s = reinterpret_cast<int*>(tslot + 1);     // chunks whose loads were issued
     int* consumed_s = issued_s + 1;                         // chunks whose MMAs were issued
 
-    // chain 1 (column chain, into W~): b = column J (B = X^T rows), t = row I (A = U_B^T rows),
-    //   K over rows I' of the source band.  chain 0 (row chain, into R, computed transposed):
-    //   b = row I (B = E rows), t = column J (A = U_A^T rows), K over columns J'.
-    // Tile (t, b) is a target when t + b lies in [tgt0, D1) (tgt0 >= mid: the band may be updated
-    // in parts); operand tile b uses K tiles [D0 - b, mid - b).  The CTA takes b0, b0 + 1 and t0, t0 + 1 and runs over the union of the
-    // two K ranges; a B box outside its own range is loaded from beyond the tensor (zeros).
+    // which tiles this CTA updates (push_cta)
     const int chain = blockIdx.z;
-    const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt, Kmax = chain ? Mt : Nt;
-    int b0, t0;
-    if constexpr (NB == 2 && MT == 2) {
-        // Target-major order (grid from push_grid_tmajor): blockIdx.y picks a slot j, a pair of
-        // target tiles, t0 = 2j + p where the pair starts one below the band edge of operand pair
-        // b0 (p = (tgt0 - 1) mod 2), t0 = 2j where that edge is clipped to 0; blockIdx.x walks the
-        // operand pairs whose band contains it.  CTAs that run together then share their U^T row
-        // slab (operand A), the larger operand of a tall or wide layer, instead of each reading
-        // its own; the set of CTAs that do work is the one of the plain (b0, t0) order.  Slots run
-        // from the highest j down: only the high slots reach the low operand pairs, whose K ranges
-        // ([D0 - b, mid - b)) are the longest, so the longest CTAs start first and the launch
-        // ends evenly.
-        const int gx = (max(Mt, Nt) + 1) / 2;
-        const int p = (tgt0 - 1) & 1;
-        const int j = (max(0, tgt0 - 1 - 2 * (gx - 1)) >> 1) + (int)(gridDim.y - 1 - blockIdx.y);
-        const int e = tgt0 - 1 - p - 2 * j;
-        b0 = 2 * ((e > 0 ? (e + 1) >> 1 : 0) + (int)blockIdx.x);
-        t0 = tgt0 - b0 - 1 > 0 ? p + 2 * j : 2 * j;
-    } else {
-        b0 = NB * blockIdx.x;
-        t0 = max(0, tgt0 - b0 - (NB - 1)) + MT * blockIdx.y;
-    }
-    if (b0 >= Bmax) return;
-    const int tlo = max(0, tgt0 - b0 - (NB - 1)), thi = min(Tmax, D1 - b0);
-    if (t0 < tlo || t0 >= thi) return;
-    const int k0 = max(0, D0 - b0 - (NB - 1)), k1 = min(Kmax, mid - b0);
-    if (k0 >= k1) return;
+    const int Bmax = chain ? Nt : Mt, Tmax = chain ? Mt : Nt;
+    PushCta cta;
+    if (!push_cta<NB, MT>((int)blockIdx.x, (int)blockIdx.y, (int)gridDim.y, chain, D0, mid, tgt0, D1, Mt, Nt, cta))
+        return;
+    const int b0 = cta.b0, t0 = cta.t0, k0 = cta.k0, k1 = cta.k1;
     grid_dep_launch();
     // set-up below overlaps the end of the previous kernel of the stream (programmatic launch);
     // everything that kernel writes -- the status word included -- is read after grid_dep_wait()

@@ -268,24 +268,19 @@ static int launch_push(const QArgs<double>& a, int D0, int mid, int tgt0, int D1
 }
 static int launch_push(const QArgs<float>& a, int D0, int mid, int tgt0, int D1, cudaStream_t st, bool pdl) {
     const int Mt = (int)a.L.Mt, Nt = (int)a.L.Nt;
-    // one CTA per (operand tiles) x (target pair): operand tile or pair of them (columns of X in the
-    // column chain, rows of E in the row chain), target pair, z = chain; pairs in target-major
-    // order (push_grid_tmajor)
+    // one CTA per (operand tiles) x (target tiles), the variant, grid and CTA order of push_variant,
+    // push_grid and push_cta
     ProfScope ps(PK_PUSH, st);
-    // pairs of operand tiles for wide bands with several target diagonals; one target diagonal
-    // (the critical part) takes one operand tile and one target tile per CTA (M = 64): beside a
-    // target on that diagonal there is no second one to fill M = 128
-    if (mid - D0 >= PUSH_PAIR_MIN_K && D1 - tgt0 > 1)
-        return launch_k(k_push_tc32<2>, push_grid_tmajor(tgt0, D1, Mt, Nt),
-                        dim3(PushCfg<2>::THREADS), PushCfg<2>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt,
-                        a.L.Np, a.Wt, a.R, *a.maps, a.status);
-    if (D1 - tgt0 == 1)
-        return launch_k(k_push_tc32<1, 1>, dim3(std::max(Mt, Nt), 1, 2), dim3(PushCfg<1, 1>::THREADS),
-                        PushCfg<1, 1>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps,
-                        a.status);
-    return launch_k(k_push_tc32<1>, dim3(std::max(Mt, Nt), (D1 - tgt0 + 1) / 2, 2), dim3(PushCfg<1>::THREADS),
-                    PushCfg<1>::SMEM_BYTES, st, pdl, D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps,
-                    a.status);
+    const int v = push_variant(D0, mid, tgt0, D1);
+    const dim3 grid = push_grid(v, tgt0, D1, Mt, Nt);
+    if (v == PV_PAIR)
+        return launch_k(k_push_tc32<2>, grid, dim3(PushCfg<2>::THREADS), PushCfg<2>::SMEM_BYTES, st, pdl, D0, mid,
+                        tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps, a.status);
+    if (v == PV_SINGLE)
+        return launch_k(k_push_tc32<1, 1>, grid, dim3(PushCfg<1, 1>::THREADS), PushCfg<1, 1>::SMEM_BYTES, st, pdl,
+                        D0, mid, tgt0, D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps, a.status);
+    return launch_k(k_push_tc32<1>, grid, dim3(PushCfg<1>::THREADS), PushCfg<1>::SMEM_BYTES, st, pdl, D0, mid, tgt0,
+                    D1, Mt, Nt, a.L.Np, a.Wt, a.R, *a.maps, a.status);
 }
 
 // ---------------------------------------------------------------------------------------
