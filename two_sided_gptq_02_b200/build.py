@@ -1,7 +1,7 @@
 """Build the kron_gptq CUDA library (libkrongptq.so) in-tree for sm_100a.
 
     python -m two_sided_gptq_02_b200.build [--force] [--verbose]
-    python -m two_sided_gptq_02_b200.build --define KG_EXPERIMENTAL_PAIR --out <path>.so
+    python -m two_sided_gptq_02_b200.build --define KG_TEST_HANDOFF_FAULT --out <path>.so
 
 Each .cu under csrc/ is compiled separately (so an unchanged file is not rebuilt) and the
 objects are linked into a shared library next to this file.  Flags: sm_100a only,
